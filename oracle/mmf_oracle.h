@@ -1,0 +1,102 @@
+/*
+ * mmf_oracle.h -- plain CPU oracle for the fused RMSNorm + BitLinear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library.  The product path (the
+ * CUDA library and its Python binding) never calls into it, and the two share
+ * no source, header, table or helper.
+ *
+ * What it computes is the definition of the BitLinear layer of the MatMul-free
+ * language model ("Scalable MatMul-free Language Modeling", Zhu et al., as
+ * described by the jiqizhixin.com article, section "具有三值权重的 MatMul-free
+ * 密集层" with its Algorithm 1 (fused RMSNorm + BitLinear), and by the
+ * datacamp.com article, section "Thay MatMul bằng các phép toán tam phân" and
+ * the "RMS norm" item of its component figure).  The pages print no formula,
+ * so every step below is the plain reading written out in each function's
+ * comment.
+ *
+ * Layouts (all row-major, no padding):
+ *   W      fp32  [N][K]   latent weights, y = x . W~^T (nn.Linear convention)
+ *   wt     int8  [N][K]   ternary weights in {-1, 0, +1}
+ *   packed uint32[N][K/16] 2-bit codes; see orc_encode_packed
+ *   x      bf16  [M][K]   activations, passed as raw uint16 bit patterns
+ *   gamma  fp32  [K]      RMSNorm gain
+ *   q      int8  [M][K]   activation codes in [-127, 127]
+ *   absmax fp32  [M]      per-token max |r| (dequantisation factor absmax/127)
+ *   acc    int32 [M][N]
+ *   y      bf16  [M][N]   raw uint16 bit patterns
+ *
+ * Error behaviour: none of these functions checks its arguments; the caller
+ * passes valid buffers of the sizes above.  The functions are sequential except
+ * orc_ternary_acc, whose outer loop over tokens may run on OpenMP threads (the
+ * result does not depend on the thread count: every acc element is a plain
+ * integer sum formed by one thread).
+ */
+#ifndef MMF_ORACLE_H
+#define MMF_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* bf16 bit pattern -> fp32 (exact). */
+float orc_bf16_to_f32(uint16_t b);
+/* fp64 -> bf16 with round-to-nearest, ties to even, computed from the
+ * definition (8 significant bits, fp32 exponent range, subnormals kept). */
+uint16_t orc_f64_to_bf16(double v);
+
+/* Absmean ternarisation (A1): beta = mean|W| summed in fp64 and rounded to
+ * fp32; wt = clamp(rint(W / (beta + eps_w)), -1, 1) with the division taken in
+ * fp32 (the precision in which the code is decided). */
+void orc_absmean_ternary(const float* W, int64_t N, int64_t K, float eps_w,
+                         int8_t* wt, float* beta);
+
+/* 2-bit packing of ternary weights (the library's storage format).
+ * K must be a multiple of 16.  Word j of row n holds weights k = 16j + i for
+ * i = 0..15; weight i sits in bits [8*(i%4) + 2*(i/4), +2) and its code is
+ * wt + 1 (0 -> -1, 1 -> 0, 2 -> +1; 3 is never written). */
+void orc_encode_packed(const int8_t* wt, int64_t N, int64_t K, uint32_t* packed);
+/* Inverse of orc_encode_packed.  Returns the number of codes equal to 3 found
+ * (which no valid packed matrix contains); those entries decode to 0. */
+int64_t orc_decode_packed(const uint32_t* packed, int64_t N, int64_t K, int8_t* wt);
+
+/* RMSNorm followed by per-token absmax int8 quantisation (A3, A4):
+ *   ms = (float)(sum_k x_k^2 / K)           sum and quotient in fp64
+ *   inv = 1 / sqrt(ms + eps)                 fp32, correctly rounded
+ *   r_k = (x_k * inv) * gamma_k              fp32, two roundings, this order
+ *   absmax = max(max_k |r_k|, 1e-5)
+ *   s = 127 / absmax                         fp32, correctly rounded
+ *   q_k = clamp(rint(r_k * s), -127, 127)    fp32 product, ties to even
+ * The fp32 part is where a float decides an integer code, so it is taken in
+ * the precision the CUDA path uses. */
+void orc_rmsnorm_quant(const uint16_t* x, const float* gamma, float eps,
+                       int64_t M, int64_t K, int8_t* q, float* absmax);
+
+/* Ternary accumulation (A2): acc[m][n] = sum over k with wt=+1 of q minus the
+ * sum over k with wt=-1 of q; a 0 weight contributes nothing.  int32. */
+void orc_ternary_acc(const int8_t* q, const int8_t* wt, int64_t M, int64_t K,
+                     int64_t N, int32_t* acc);
+
+/* Rescale (A5): y = bf16_rn(acc * (absmax / 127) * beta), evaluated in fp64
+ * and rounded once to bf16. */
+void orc_rescale(const int32_t* acc, const float* absmax, float beta,
+                 int64_t M, int64_t N, uint16_t* y);
+
+/* The whole layer from latent weights: ternarise W, quantise x, accumulate,
+ * rescale.  Scratch for wt (N*K bytes), q (M*K bytes), absmax (M floats) and
+ * acc (M*N int32) is allocated and freed inside.  Returns 0, or -1 if an
+ * allocation failed. */
+int orc_bitlinear(const uint16_t* x, const float* gamma, float eps,
+                  const float* W, float eps_w, int64_t M, int64_t K, int64_t N,
+                  uint16_t* y, float* beta_out);
+
+/* Number of OpenMP threads orc_ternary_acc uses (1 when built without OpenMP). */
+int orc_num_threads(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MMF_ORACLE_H */
