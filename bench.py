@@ -1,0 +1,479 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused RMSNorm + BitLinear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--layers L]
+
+Prints ONE JSON line (rank 0).  Default workload: decode at the 2.7B width,
+M = 1 token, the 7-projection BitLinear set (4x 2560->2560, 2x 2560->6912,
+6912->2560), repeated over L = 32 layer sets with distinct weights so the
+packed weights (634 MB) exceed L2 and stream from HBM every step.
+
+A step = one pass of the whole hot path (RMSNorm, int8 quantisation, ternary
+contraction, rescale: every projection of every layer set) over one batch of M
+tokens, replayed as one CUDA graph.  `value` = tokens/s through one layer set
+(M * L * n_gpus / step time), i.e. the decode rate of one token through the
+BitLinear set of one layer.  Weights are packed once, before timing (offline
+on the pages' terms).
+
+--impl reference times the CPU oracle (the only reference this method has on
+the box), on bounded samples of the same workload.  Multi-GPU: one process per
+GPU (torchrun), token-parallel replicas with no data-path collective; a
+barrier and a MAX all-reduce of the device-timed step time only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bitlinear_rmsnorm_quant_b200 import inputs as I  # noqa: E402
+from bitlinear_rmsnorm_quant_b200 import workloads as WL  # noqa: E402
+
+METRIC = "fused RMSNorm+BitLinear tokens/s; GB/s or int8 TOPS as % of B200 roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_PER_BF16 = 2.0   # nominal dense ratio int8 : bf16 (4.5 : 2.25 POPS)
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ----------------------------------------------------------------------------- dist
+
+class Dist:
+    def __init__(self, gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import torch.distributed as dist
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local_rank)
+            import datetime
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+        if gpus != self.world:
+            raise SystemExit(f"--gpus {gpus} but WORLD_SIZE={self.world}")
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if self.pg is None:
+            return v
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML during the timed region."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x10: "sync_boost", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.ok = False
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            self.N = N
+            try:
+                p = torch.cuda.get_device_properties(device_index)
+                bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+                self.h = N.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = N.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def _read(self):
+        N = self.N
+        self.samples.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+        try:
+            self.reasons |= int(N.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+        except Exception:
+            self.reasons |= int(N.nvmlDeviceGetCurrentClocksThrottleReasons(self.h))
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                self._read()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._loop, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+            try:
+                self._read()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [v for k, v in self.REASONS.items() if self.reasons & k and v != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+WORKLOADS = {
+    "decode-2.7b-m1": (lambda: WL.decode_2p7b(1), 32),
+    "decode-2.7b-m8": (lambda: WL.decode_2p7b(8), 32),
+    "decode-2.7b-m32": (lambda: WL.decode_2p7b(32), 32),
+    "decode-370m": (lambda: WL.DECODE_370M, 160),
+    "prefill-1.3b": (lambda: WL.PREFILL_1P3B, 1),
+    "train-fwd-1.3b": (lambda: WL.TRAIN_FWD_1P3B, 1),
+    "smoke-256": (lambda: WL.SMOKE, 1),
+}
+DEFAULT_WORKLOAD = "decode-2.7b-m1"
+
+
+def proj_bytes(M, K, N):
+    """Algorithmic HBM bytes of one fused BitLinear call: packed W, x, gamma, y, beta."""
+    return N * K // 4 + 2 * M * K + 4 * K + 2 * M * N + 4
+
+
+def proj_ops(M, K, N):
+    return 2 * M * N * K
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, dist: Dist):
+    from bitlinear_rmsnorm_quant_b200 import mmf
+    dev = torch.device("cuda", dist.local_rank)
+    torch.cuda.set_device(dev)
+    wl, default_layers = WORKLOADS[args.workload]
+    wl = wl()
+    L = args.layers or default_layers
+    M = wl.M
+    seed = wl.seed + 7919 * dist.rank  # each rank draws its own tokens and weights
+
+    # -- weights: drawn on the device, packed once (offline), fp32 freed
+    packed, scales = {}, {}
+    for l in range(L):
+        for j, p in enumerate(wl.projections):
+            W = I.latent_weights(seed, p.N, p.K, index=64 * l + j, device=dev)
+            packed[l, j], scales[l, j] = mmf.pack_ternary(W, wl.eps_w)
+            del W
+    # -- activations and outputs: views into one flat device buffer each, so the
+    #    end-to-end step is one H2D copy, the graph, and one D2H copy
+    def carve(shapes):
+        offs, total = [], 0
+        for shp in shapes:
+            offs.append(total)
+            total += (math.prod(shp) + 7) // 8 * 8      # 16-byte aligned views
+        flat = torch.empty(max(total, 8), dtype=torch.bfloat16, device=dev)
+        return flat, [flat[o:o + math.prod(shp)].view(*shp) for o, shp in zip(offs, shapes)]
+
+    x_keys = [(l, idx) for l in range(L) for idx, _ in wl.inputs()]
+    x_flat, x_views = carve([(M, dict(wl.inputs())[idx]) for _, idx in x_keys])
+    xs = dict(zip(x_keys, x_views))
+    for (l, idx), xv in xs.items():
+        xv.copy_(I.activations(seed, M, xv.shape[1], index=64 * l + idx, outlier_frac=wl.outlier_frac, device=dev))
+    gs = {(l, idx): I.gamma(seed, K, index=64 * l + idx, device=dev) for l in range(L) for idx, K in wl.inputs()}
+    y_keys = [(l, j) for l in range(L) for j in range(len(wl.projections))]
+    y_flat, y_views = carve([(M, wl.projections[j].N) for _, j in y_keys])
+    ys = dict(zip(y_keys, y_views))
+    ws_need = max(mmf.workspace_bytes(M, p.K, p.N) for p in wl.projections)
+    ws = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=dev)
+    lib = mmf.lib()
+
+    calls = []
+    launches_per_step = 0
+    bytes_per_step = 0
+    ops_per_step = 0
+    for l in range(L):
+        for j, p in enumerate(wl.projections):
+            x, g = xs[l, p.input_index], gs[l, p.input_index]
+            calls.append((x.data_ptr(), g.data_ptr(), wl.eps, packed[l, j].data_ptr(), scales[l, j].data_ptr(),
+                          M, p.K, p.N, ys[l, j].data_ptr(), ws.data_ptr(), ws.numel()))
+            launches_per_step += 1 if mmf.workspace_bytes(M, p.K, p.N) == 0 else 2
+            bytes_per_step += proj_bytes(M, p.K, p.N)
+            ops_per_step += proj_ops(M, p.K, p.N)
+    decode_path = all(mmf.workspace_bytes(M, p.K, p.N) == 0 for p in wl.projections)
+
+    def step(stream_ptr):
+        for c in calls:
+            rc = lib.mmf_bitlinear_fwd(*c, stream_ptr)
+            if rc != 0:
+                raise mmf.MMFError("mmf_bitlinear_fwd", rc)
+
+    # first calls outside capture (one-time per-device set-up), then capture
+    step(torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    mmf.check_async()
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    with torch.cuda.stream(cap):
+        graph.capture_begin()
+        step(cap.cuda_stream)
+        graph.capture_end()
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    mmf.check_async()
+
+    # -- timed region: K graph replays, CUDA events on the replay stream
+    clocks = ClockSampler(dist.local_rank)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0.record()
+    for _ in range(args.steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks.stop()
+    dist.barrier()
+    ms_local = e0.elapsed_time(e1) / args.steps
+    mmf.check_async()
+    ms = dist.max(ms_local)
+
+    # -- end to end: pinned host x -> device, the graph (the ABI calls), y -> pinned host
+    h_x = x_flat.cpu().pin_memory()
+    h_y = torch.empty(y_flat.shape, dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        x_flat.copy_(h_x, non_blocking=True)
+        graph.replay()
+        h_y.copy_(y_flat, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 200))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    e2e_ms = dist.max(f0.elapsed_time(f1) / e2e_steps)
+
+    tokens_per_step = M * L * dist.world
+    value = tokens_per_step / (ms / 1e3)
+    e2e_value = tokens_per_step / (e2e_ms / 1e3)
+
+    peaks, peak_src = load_peaks()
+    if decode_path:
+        achieved = bytes_per_step / (ms / 1e3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": None, "kernel": "gemv_kernel",
+                "peak_source": f"{peak_src} hbm_gbs (copy of 1 Gi bf16, read+write bytes)",
+                "algorithmic_bytes_per_step": bytes_per_step,
+                "note": "step time over all launches, inter-kernel gaps included"}
+    else:
+        achieved = ops_per_step / (ms / 1e3) / 1e12
+        peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None, "kernel": "gemm_tc_kernel",
+                "peak_source": f"{peak_src} bf16_tflops x {INT8_PER_BF16} (nominal int8:bf16 dense ratio)",
+                "algorithmic_ops_per_step": ops_per_step,
+                "note": "int8 TOPS over the whole step (quantiser kernel included)"}
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "tokens/s (one token through one BitLinear layer set)",
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic (seeded SplitMix64/Box-Muller; random-init latent weights)",
+        "config": {
+            "workload": wl.name, "description": wl.description, "M": M, "layer_sets": L,
+            "projections": [f"{p.K}->{p.N}" for p in wl.projections],
+            "packed_weight_bytes": sum(p.N * p.K // 4 for p in wl.projections) * L,
+            "l2": "inputs larger than L2: packed weights of all layer sets exceed 126 MB"
+                  if sum(p.N * p.K // 4 for p in wl.projections) * L > L2_BYTES else "working set below L2",
+            "graph": "one CUDA graph per step", "parallelism": f"dp{dist.world} (token-parallel replicas)",
+        },
+        "roofline": roof,
+        "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s (one token through one BitLinear layer set)",
+                "h2d_bytes_per_step": int(h_x.numel() * 2), "d2h_bytes_per_step": int(h_y.numel() * 2),
+                "steps": e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    del graph
+    return result, wl, L
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def time_oracle(wl, sample_tokens: int | None, budget_s: float, max_reps: int | None = None,
+                one_projection_per_rep: bool = False):
+    """Times the CPU oracle (ternarised weights prepared untimed) on a bounded
+    sample: rmsnorm+quant, ternary accumulation and rescale for each projection."""
+    import numpy as np
+
+    from oracle import load
+    orc = load()
+    M = wl.M if sample_tokens is None else min(wl.M, sample_tokens)
+    prep = []
+    for j, p in enumerate(wl.projections):
+        W = I.latent_weights(wl.seed, p.N, p.K, index=j).numpy()
+        wt, beta = orc.absmean_ternary(W, wl.eps_w)
+        x = I.activations(wl.seed, M, p.K, index=p.input_index, outlier_frac=wl.outlier_frac)
+        xb = x.view(torch.int16).numpy().view(np.uint16)
+        g = I.gamma(wl.seed, p.K, index=p.input_index).numpy()
+        prep.append((xb, g, wt, beta))
+    per_proj = [[] for _ in prep]
+    t_start = time.perf_counter()
+    reps = 0
+    while True:
+        todo = [reps % len(prep)] if one_projection_per_rep else range(len(prep))
+        for j in todo:
+            xb, g, wt, beta = prep[j]
+            t0 = time.perf_counter()
+            q, a = orc.rmsnorm_quant(xb, g, wl.eps)
+            acc = orc.ternary_acc(q, wt)
+            orc.rescale(acc, a, beta)
+            per_proj[j].append(time.perf_counter() - t0)
+        reps += 1
+        if max_reps is not None and reps >= max_reps and all(per_proj):
+            break
+        if time.perf_counter() - t_start > budget_s and all(per_proj):
+            break
+    t_set = sum(statistics.median(v) for v in per_proj)
+    threads = min(orc.num_threads(), M)
+    return M / t_set, M, threads, reps
+
+
+def oracle_sample_tokens(wl, cap):
+    return cap if wl.M > cap else None
+
+
+def cpu_baseline_obj(wl, budget_s=12.0):
+    sample = oracle_sample_tokens(wl, 512)
+    tps, M, threads, reps = time_oracle(wl, sample, budget_s)
+    return {"value": round(tps, 3), "unit": "tokens/s (one token through one BitLinear layer set)",
+            "cores": threads, "kind": "oracle",
+            "sample": f"{M} tokens x all {len(wl.projections)} projections, median of {reps} rep(s), "
+                      f"OpenMP over tokens; weights ternarised untimed"
+                      + (f"; extrapolated linearly from {M} of {wl.M} tokens" if M < wl.M else "")}
+
+
+def run_reference(args, dist: Dist):
+    wl, _ = WORKLOADS[args.workload]
+    wl = wl()
+    if dist.rank != 0:
+        return None
+    sample = oracle_sample_tokens(wl, 64)
+    # each step: one projection of the set (round robin) on the sampled tokens;
+    # the run stops after --steps steps or 150 s, whichever comes first
+    t0 = time.perf_counter()
+    tps, M, threads, reps = time_oracle(wl, sample, budget_s=150.0, max_reps=max(args.steps, len(wl.projections)),
+                                        one_projection_per_rep=True)
+    wall = time.perf_counter() - t0
+    ms_per_step = 1e3 * M / tps / len(wl.projections)
+    return {
+        "metric": METRIC, "impl": "reference", "value": round(tps, 3),
+        "unit": "tokens/s (one token through one BitLinear layer set)",
+        "n_gpus": dist.world, "steps": reps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded SplitMix64/Box-Muller; random-init latent weights)",
+        "config": {"workload": wl.name, "description": wl.description, "M": wl.M,
+                   "projections": [f"{p.K}->{p.N}" for p in wl.projections]},
+        "cpu_baseline": {"value": round(tps, 3), "unit": "tokens/s (one token through one BitLinear layer set)",
+                         "cores": threads, "kind": "oracle",
+                         "sample": f"{M} tokens; each step one projection (round robin); wall {wall:.1f} s"},
+        "e2e": {"value": round(tps, 3), "unit": "tokens/s (one token through one BitLinear layer set)",
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--layers", type=int, default=0, help="layer sets per step (default per workload)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    dist = Dist(args.gpus)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, dist)
+            if res is not None:
+                print(json.dumps(res), flush=True)
+            return 0
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py --impl ours needs a CUDA device")
+        res, wl, L = run_ours(args, dist)
+        if dist.rank == 0:
+            if dist.world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline_obj(wl)
+            print(json.dumps(res), flush=True)
+        return 0
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

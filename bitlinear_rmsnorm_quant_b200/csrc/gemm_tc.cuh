@@ -1,0 +1,227 @@
+// gemm_tc.cuh -- large-M ternary contraction on the 5th-generation tensor
+// cores (tcgen05, kind::i8, int32 accumulators in TMEM).
+//
+// The product with ternary weights is a dense contraction at large M, so it
+// runs as one: the 2-bit weight codes c = w~ + 1 are unpacked to int8 in
+// shared memory and multiplied with the int8 activation codes; the epilogue
+// subtracts the per-token sum of q, which turns sum_k c q into
+// sum_k w~ q = (sum over w~=+1 of q) - (sum over w~=-1 of q)
+// (the ternary accumulation of ld246.com, section "三值权重的应用").
+//
+// Tile: 128 weight rows (MMA M) x BT tokens (MMA N) x 128 K per stage; the
+// weights are the A operand, so one unpacked weight tile feeds BT tokens.
+// Warp roles (256 threads):
+//   warp 0      TMA producer: q tile (BT x 128 B, 128-byte swizzle) and the
+//               packed weight tile (128 x 32 B) per stage
+//   warp 1      TMEM allocation; lane 0 issues tcgen05.mma (4 x K=32 per
+//               stage) and tcgen05.commit
+//   warps 4-7   unpack: thread u expands row u's 128 codes to int8 in the
+//               128-byte-swizzled K-major layout the MMA reads; then the
+//               epilogue (tcgen05.ld, subtract qsum, rescale, store)
+// Every wait is bounded; on timeout the CTA records the error, drains its
+// copies and MMAs, frees TMEM and exits.
+#pragma once
+#include "common.cuh"
+
+namespace mmf {
+
+constexpr int kTcRows = 128;      // weight rows per tile (MMA M)
+constexpr int kTcK = 128;         // K (bytes of int8) per stage
+constexpr int kTcStages = 4;
+constexpr int kTcThreads = 256;
+constexpr int kTcPackedBytes = kTcRows * (kTcK / 4);  // 4 KB of 2-bit codes per stage
+
+template <int BT>
+struct TcLayout {
+    static constexpr int a_bytes = kTcRows * kTcK;  // 16 KB
+    static constexpr int b_bytes = BT * kTcK;
+    static constexpr int stage_bytes = a_bytes + b_bytes + kTcPackedBytes;
+    static constexpr int smem_bytes = kTcStages * stage_bytes + 1024;  // + alignment slack
+    static constexpr int tmem_cols = BT < 32 ? 32 : BT;
+};
+
+struct TcParams {
+    const int8_t* q;        // unused by the kernel body (read through the tensor map)
+    const int* qsum;        // [M]
+    const float* absmax;    // [M]      (fused mode)
+    const float* scale;     // beta     (fused mode)
+    uint16_t* y;            // bf16 [M][N]
+    int32_t* acc;           // int32 [M][N]
+    int M, K, N;
+};
+
+template <int BT, bool FUSED>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_w,
+                   const TcParams p) {
+    using L = TcLayout<BT>;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[kTcStages];
+    __shared__ __align__(8) uint64_t unpacked_bar[kTcStages];
+    __shared__ __align__(8) uint64_t empty_bar[kTcStages];
+    __shared__ __align__(8) uint64_t accfull_bar;
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_flag;
+    __shared__ int qsum_s[BT];
+    __shared__ float cm_s[BT];
+
+    // 1024-byte aligned base (128-byte swizzle atoms are 8 rows x 128 B)
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    auto a_tile = [&](int s) { return smem + s * L::stage_bytes; };
+    auto b_tile = [&](int s) { return smem + s * L::stage_bytes + L::a_bytes; };
+    auto p_tile = [&](int s) { return smem + s * L::stage_bytes + L::a_bytes + L::b_bytes; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * kTcRows;
+    const int t0 = blockIdx.y * BT;
+    const int nk = p.K / kTcK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&unpacked_bar[s], 128);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&accfull_bar, 1);
+        mbar_init(&drain_bar, 1);
+        abort_flag = 0;
+        mbar_fence_init();
+        prefetch_tensormap(&tmap_q);
+        prefetch_tensormap(&tmap_w);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_s, L::tmem_cols);
+        tmem_relinquish();
+    }
+    if (warp >= 4) {
+        // per-token epilogue constants of this tile
+        for (int i = threadIdx.x - 128; i < BT; i += 128) {
+            const int t = t0 + i;
+            int qs = 0;
+            float cm = 0.0f;
+            if (t < p.M) {
+                qs = p.qsum[t];
+                if constexpr (FUSED) cm = __fmul_rn(__fdiv_rn(p.absmax[t], 127.0f), __ldg(p.scale));
+            }
+            qsum_s[i] = qs;
+            cm_s[i] = cm;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_acc = tmem_base_s;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int ks = 0; ks < nk; ++ks) {
+                const int s = ks % kTcStages;
+                if (ks >= kTcStages && !mbar_wait(&empty_bar[s], ((ks / kTcStages) - 1) & 1, &abort_flag)) break;
+                mbar_arrive_expect_tx(&full_bar[s], L::b_bytes + kTcPackedBytes);
+                tma_load_2d(b_tile(s), &tmap_q, ks * kTcK, t0, &full_bar[s]);
+                tma_load_2d(p_tile(s), &tmap_w, ks * (kTcK / 4), n0, &full_bar[s]);
+                ++issued;
+            }
+            int zero = 0;
+            for (int ks = max(0, issued - kTcStages); ks < issued; ++ks)
+                mbar_wait(&full_bar[ks % kTcStages], (ks / kTcStages) & 1, &zero);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_i8(kTcRows, BT);
+            bool issued_any = false;
+            for (int ks = 0; ks < nk; ++ks) {
+                const int s = ks % kTcStages;
+                const uint32_t par = (ks / kTcStages) & 1;
+                if (!mbar_wait(&full_bar[s], par, &abort_flag)) break;
+                if (!mbar_wait(&unpacked_bar[s], par, &abort_flag)) break;
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(a_tile(s)), b0 = smem_u32(b_tile(s));
+#pragma unroll
+                for (int kk = 0; kk < kTcK / 32; ++kk) {
+                    mma_i8(tmem_acc, sw128_kmajor_desc(a0 + 32 * kk), sw128_kmajor_desc(b0 + 32 * kk), idesc,
+                           (ks | kk) != 0 ? 1u : 0u);
+                }
+                issued_any = true;
+                mma_commit(&empty_bar[s]);
+            }
+            if (!abort_flag) mma_commit(&accfull_bar);
+            if (issued_any) {
+                mma_commit(&drain_bar);
+                int zero = 0;
+                mbar_wait(&drain_bar, 0, &zero);
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ unpack
+        const int u = threadIdx.x - 128;  // weight row within the tile
+        for (int ks = 0; ks < nk; ++ks) {
+            const int s = ks % kTcStages;
+            if (!mbar_wait(&full_bar[s], (ks / kTcStages) & 1, &abort_flag)) break;
+            const uint4* prow = reinterpret_cast<const uint4*>(p_tile(s) + u * (kTcK / 4));
+            const uint4 pa = prow[0], pb = prow[1];
+            const uint32_t words[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+            uint8_t* arow = a_tile(s) + (u >> 3) * 1024 + (u & 7) * 128;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                // word t holds K bytes 16t .. 16t+15 of this stage; byte-lane j of
+                // the output chunk gets codes 4j .. 4j+3 (bits 2j of each byte)
+                const uint32_t w = words[t];
+                uint4 o;
+                o.x = w & 0x03030303u;
+                o.y = (w >> 2) & 0x03030303u;
+                o.z = (w >> 4) & 0x03030303u;
+                o.w = (w >> 6) & 0x03030303u;
+                *reinterpret_cast<uint4*>(arow + ((t ^ (u & 7)) << 4)) = o;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&unpacked_bar[s]);
+        }
+
+        // ------------------------------------------------------------ epilogue
+        const int wq = warp - 4;  // TMEM lanes 32*wq .. 32*wq+31
+        const int n = n0 + 32 * wq + lane;
+        const bool ok = mbar_wait(&accfull_bar, 0, &abort_flag);
+        tc_fence_after();
+        if (ok) {
+#pragma unroll 1
+            for (int cc = 0; cc < BT / 32 || (BT < 32 && cc == 0); ++cc) {
+                uint32_t r[32];
+                const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(32 * wq) << 16) + 32 * cc;
+                tmem_ld_32x32b_x32(taddr, r);
+                tmem_ld_wait();
+                if (n < p.N) {
+                    const int ncols = BT < 32 ? BT : 32;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        if (i >= ncols) break;
+                        const int ti = 32 * cc + i;
+                        const int t = t0 + ti;
+                        if (t < p.M) {
+                            const int v = static_cast<int>(r[i]) - qsum_s[ti];
+                            if constexpr (FUSED) {
+                                const __nv_bfloat16 yb = __float2bfloat16_rn(__fmul_rn(static_cast<float>(v), cm_s[ti]));
+                                p.y[static_cast<size_t>(t) * p.N + n] = __bfloat16_as_ushort(yb);
+                            } else {
+                                p.acc[static_cast<size_t>(t) * p.N + n] = v;
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_acc, L::tmem_cols);
+    }
+}
+
+}  // namespace mmf

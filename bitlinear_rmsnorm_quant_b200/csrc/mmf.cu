@@ -1,0 +1,415 @@
+// mmf.cu -- the C ABI of libmmf.so (declared in include/mmf.h): argument
+// checks, kernel dispatch by M, tensor-map construction.  All kernels live in
+// the headers included below; this is the only translation unit.
+#include "mmf.h"
+
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "copy.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "pack.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using namespace mmf;
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+constexpr int64_t kMaxK = 65536;  // the quantiser stages one bf16 row (2K bytes) in shared memory
+
+struct DeviceState {
+    bool ready = false;
+    int num_sms = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+template <typename F>
+cudaError_t set_smem(F* f, size_t bytes) {
+    return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+}
+
+template <int BT>
+cudaError_t set_tc_attrs() {
+    cudaError_t e = set_smem(gemm_tc_kernel<BT, true>, TcLayout<BT>::smem_bytes);
+    if (e == cudaSuccess) e = set_smem(gemm_tc_kernel<BT, false>, TcLayout<BT>::smem_bytes);
+    return e;
+}
+
+template <int MT>
+cudaError_t set_gemv_attrs() {
+    cudaError_t e = set_smem(gemv_kernel<MT, true>, 200 * 1024);
+    if (e == cudaSuccess) e = set_smem(gemv_kernel<MT, false>, 200 * 1024);
+    return e;
+}
+
+// Per-device one-time set-up (device properties, kernel attributes, the driver
+// entry point for tensor maps).  Must run before any stream capture.
+mmf_status device_state(DeviceState** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MMF_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& st = g_dev[dev];
+    if (!st.ready) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MMF_ERR_CUDA;
+        if (prop.major != 10) return MMF_ERR_NO_DEVICE;
+        st.num_sms = prop.multiProcessorCount;
+        cudaError_t e = cudaSuccess;
+        if (e == cudaSuccess) e = set_tc_attrs<16>();
+        if (e == cudaSuccess) e = set_tc_attrs<32>();
+        if (e == cudaSuccess) e = set_tc_attrs<64>();
+        if (e == cudaSuccess) e = set_tc_attrs<128>();
+        if (e == cudaSuccess) e = set_tc_attrs<256>();
+        if (e == cudaSuccess) e = set_gemv_attrs<1>();
+        if (e == cudaSuccess) e = set_gemv_attrs<2>();
+        if (e == cudaSuccess) e = set_gemv_attrs<3>();
+        if (e == cudaSuccess) e = set_gemv_attrs<4>();
+        if (e == cudaSuccess) e = set_gemv_attrs<5>();
+        if (e == cudaSuccess) e = set_gemv_attrs<6>();
+        if (e == cudaSuccess) e = set_gemv_attrs<7>();
+        if (e == cudaSuccess) e = set_gemv_attrs<8>();
+        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel, 2 * kMaxK);
+        if (e != cudaSuccess) return MMF_ERR_CUDA;
+        if (!g_encode_tiled) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                return MMF_ERR_CUDA;
+            g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        st.ready = true;
+    }
+    *out = &st;
+    return MMF_OK;
+}
+
+inline mmf_status launch_status() { return cudaGetLastError() == cudaSuccess ? MMF_OK : MMF_ERR_CUDA; }
+
+mmf_status check_shape(int64_t M, int64_t K, int64_t N) {
+    if (M < 0 || N < 0 || K < 0) return MMF_ERR_INVALID_ARG;
+    if (K < 128 || (K % 128) != 0 || K > kMaxK) return MMF_ERR_UNSUPPORTED_SHAPE;
+    if (M > kMaxDim || N > kMaxDim) return MMF_ERR_UNSUPPORTED_SHAPE;
+    if (M > int64_t(65535) * 256) return MMF_ERR_UNSUPPORTED_SHAPE;  // token tiles on grid.y
+    if (M * K > (int64_t(1) << 40) || N * K > (int64_t(1) << 40)) return MMF_ERR_UNSUPPORTED_SHAPE;
+    return MMF_OK;
+}
+
+bool takes_gemv(int64_t M, int64_t K, int64_t N) {
+    GemvPlan plan;
+    return gemv_plan(static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), 148, &plan);
+}
+
+int token_tile(int64_t M) {
+    if (M <= 16) return 16;
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return 256;
+}
+
+struct Workspace {
+    int8_t* q;
+    float* absmax;
+    int* qsum;
+};
+
+size_t workspace_size_tc(int64_t M, int64_t K) {
+    return align256(static_cast<size_t>(M) * K) + 2 * align256(4 * static_cast<size_t>(M));
+}
+
+Workspace carve(void* ws, int64_t M, int64_t K) {
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    Workspace w;
+    w.q = reinterpret_cast<int8_t*>(b);
+    w.absmax = reinterpret_cast<float*>(b + align256(static_cast<size_t>(M) * K));
+    w.qsum = reinterpret_cast<int*>(b + align256(static_cast<size_t>(M) * K) + align256(4 * static_cast<size_t>(M)));
+    return w;
+}
+
+mmf_status make_maps(const int8_t* q, const uint32_t* packed, int64_t M, int64_t K, int64_t N, int BT,
+                     CUtensorMap* mq, CUtensorMap* mw) {
+    const cuuint32_t es[2] = {1, 1};
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcK), static_cast<cuuint32_t>(BT)};
+        if (g_encode_tiled(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(q), dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MMF_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 4), static_cast<cuuint64_t>(N)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 4)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcK / 4), static_cast<cuuint32_t>(kTcRows)};
+        if (g_encode_tiled(mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint32_t*>(packed), dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MMF_ERR_CUDA;
+    }
+    return MMF_OK;
+}
+
+template <int BT>
+mmf_status launch_tc_bt(bool fused, const CUtensorMap& mq, const CUtensorMap& mw, const TcParams& p,
+                        cudaStream_t s) {
+    const dim3 grid(static_cast<unsigned>((p.N + kTcRows - 1) / kTcRows), static_cast<unsigned>((p.M + BT - 1) / BT));
+    if (fused)
+        gemm_tc_kernel<BT, true><<<grid, kTcThreads, TcLayout<BT>::smem_bytes, s>>>(mq, mw, p);
+    else
+        gemm_tc_kernel<BT, false><<<grid, kTcThreads, TcLayout<BT>::smem_bytes, s>>>(mq, mw, p);
+    return launch_status();
+}
+
+mmf_status launch_tc(bool fused, const int8_t* q, const uint32_t* packed, const TcParams& p, cudaStream_t s) {
+    const int BT = token_tile(p.M);
+    CUtensorMap mq, mw;
+    mmf_status st = make_maps(q, packed, p.M, p.K, p.N, BT, &mq, &mw);
+    if (st != MMF_OK) return st;
+    switch (BT) {
+        case 16: return launch_tc_bt<16>(fused, mq, mw, p, s);
+        case 32: return launch_tc_bt<32>(fused, mq, mw, p, s);
+        case 64: return launch_tc_bt<64>(fused, mq, mw, p, s);
+        case 128: return launch_tc_bt<128>(fused, mq, mw, p, s);
+        default: return launch_tc_bt<256>(fused, mq, mw, p, s);
+    }
+}
+
+template <bool FUSED>
+mmf_status launch_gemv(const GemvParams& p, const GemvPlan& plan, cudaStream_t s) {
+    const dim3 grid(static_cast<unsigned>(plan.grid));
+    switch (p.M) {
+#define MMF_GEMV_CASE(MT) \
+    case MT: gemv_kernel<MT, FUSED><<<grid, kGemvThreads, plan.smem_bytes, s>>>(p); break;
+        MMF_GEMV_CASE(1)
+        MMF_GEMV_CASE(2)
+        MMF_GEMV_CASE(3)
+        MMF_GEMV_CASE(4)
+        MMF_GEMV_CASE(5)
+        MMF_GEMV_CASE(6)
+        MMF_GEMV_CASE(7)
+        MMF_GEMV_CASE(8)
+#undef MMF_GEMV_CASE
+        default: return MMF_ERR_UNSUPPORTED_SHAPE;
+    }
+    return launch_status();
+}
+
+mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K, int8_t* q,
+                        float* absmax, int* qsum, cudaStream_t s) {
+    const size_t smem = static_cast<size_t>(K) * 2;
+    rmsnorm_quant_kernel<<<static_cast<unsigned>(M), kQuantThreads, smem, s>>>(x, gamma, eps, static_cast<int>(K), q,
+                                                                                absmax, qsum);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mmf_status_string(int status) {
+    switch (status) {
+        case MMF_OK: return "MMF_OK";
+        case MMF_ERR_INVALID_ARG: return "MMF_ERR_INVALID_ARG";
+        case MMF_ERR_UNSUPPORTED_SHAPE: return "MMF_ERR_UNSUPPORTED_SHAPE";
+        case MMF_ERR_MISALIGNED: return "MMF_ERR_MISALIGNED";
+        case MMF_ERR_WORKSPACE: return "MMF_ERR_WORKSPACE";
+        case MMF_ERR_CUDA: return "MMF_ERR_CUDA";
+        case MMF_ERR_TIMEOUT: return "MMF_ERR_TIMEOUT";
+        case MMF_ERR_NO_DEVICE: return "MMF_ERR_NO_DEVICE";
+        default: return "MMF_ERR_UNKNOWN";
+    }
+}
+
+const char* mmf_version(void) { return "mmf 0.1.0 sm_100a"; }
+
+size_t mmf_packed_bytes(int64_t N, int64_t K) {
+    if (N < 0 || K < 0) return 0;
+    return static_cast<size_t>(N) * static_cast<size_t>(K) / 4;
+}
+
+size_t mmf_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+    if (check_shape(M, K, N) != MMF_OK || M == 0 || N == 0) return 0;
+    if (takes_gemv(M, K, N)) return 0;
+    return workspace_size_tc(M, K);
+}
+
+int mmf_pack_ternary(const float* W, int64_t N, int64_t K, float eps_w, uint32_t* packed, float* scale,
+                     void* stream) {
+    if (!W || !packed || !scale) return MMF_ERR_INVALID_ARG;
+    if (!(eps_w >= 0.0f) || eps_w > 1e30f) return MMF_ERR_INVALID_ARG;
+    mmf_status st = check_shape(0, K, N);
+    if (st != MMF_OK) return st;
+    if (!aligned16(W) || !aligned16(packed) || !aligned16(scale)) return MMF_ERR_MISALIGNED;
+    if (N == 0) return MMF_OK;
+    DeviceState* dev;
+    if ((st = device_state(&dev)) != MMF_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t n = N * K;
+    const int np = absmean_num_partials(n);
+    int64_t chunk = (n + np - 1) / np;
+    chunk = (chunk + 3) & ~int64_t(3);
+    double* partials = reinterpret_cast<double*>(packed);  // scratch: the codes overwrite it below
+    absmean_partials_kernel<<<np, kPackThreads, 0, s>>>(W, n, chunk, partials);
+    if ((st = launch_status()) != MMF_OK) return st;
+    absmean_finalize_kernel<<<1, kPackThreads, 0, s>>>(partials, np, n, scale);
+    if ((st = launch_status()) != MMF_OK) return st;
+    const int64_t nwords = n / 16;
+    int64_t grid = (nwords + kPackThreads - 1) / kPackThreads;
+    if (grid > int64_t(dev->num_sms) * 16) grid = int64_t(dev->num_sms) * 16;
+    ternary_encode_kernel<<<static_cast<unsigned>(grid), kPackThreads, 0, s>>>(W, nwords, eps_w, scale, packed);
+    return launch_status();
+}
+
+int mmf_quantize_act(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K, int8_t* q,
+                     float* absmax, void* stream) {
+    if (!x || !gamma || !q || !absmax) return MMF_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || eps > 1e30f) return MMF_ERR_INVALID_ARG;
+    mmf_status st = check_shape(M, K, 1);
+    if (st != MMF_OK) return st;
+    if (!aligned16(x) || !aligned16(gamma) || !aligned16(q) || !aligned16(absmax)) return MMF_ERR_MISALIGNED;
+    if (M == 0) return MMF_OK;
+    DeviceState* dev;
+    if ((st = device_state(&dev)) != MMF_OK) return st;
+    return launch_quant(x, gamma, eps, M, K, q, absmax, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t K, int64_t N, int32_t* acc,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q || !packed || !acc) return MMF_ERR_INVALID_ARG;
+    mmf_status st = check_shape(M, K, N);
+    if (st != MMF_OK) return st;
+    if (!aligned16(q) || !aligned16(packed) || !aligned16(acc)) return MMF_ERR_MISALIGNED;
+    if (M == 0 || N == 0) return MMF_OK;
+    const size_t need = mmf_workspace_bytes(M, K, N);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return MMF_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return MMF_ERR_MISALIGNED;
+    DeviceState* dev;
+    if ((st = device_state(&dev)) != MMF_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    GemvPlan plan;
+    if (gemv_plan(static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), dev->num_sms, &plan)) {
+        GemvParams p{};
+        p.q_in = q;
+        p.packed = packed;
+        p.acc = acc;
+        p.M = static_cast<int>(M);
+        p.K = static_cast<int>(K);
+        p.N = static_cast<int>(N);
+        p.rows_per_stage = plan.rows_per_stage;
+        p.rows_per_cta = plan.rows_per_cta;
+        p.stage_bytes = plan.stage_bytes;
+        return launch_gemv<false>(p, plan, s);
+    }
+    Workspace w = carve(workspace, M, K);
+    qsum_kernel<<<static_cast<unsigned>(M), kQuantThreads, 0, s>>>(q, static_cast<int>(K), w.qsum);
+    if ((st = launch_status()) != MMF_OK) return st;
+    TcParams p{};
+    p.qsum = w.qsum;
+    p.acc = acc;
+    p.M = static_cast<int>(M);
+    p.K = static_cast<int>(K);
+    p.N = static_cast<int>(N);
+    return launch_tc(false, q, packed, p, s);
+}
+
+int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps, const uint32_t* packed, const float* scale,
+                      int64_t M, int64_t K, int64_t N, uint16_t* y, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+    if (!x || !gamma || !packed || !scale || !y) return MMF_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || eps > 1e30f) return MMF_ERR_INVALID_ARG;
+    mmf_status st = check_shape(M, K, N);
+    if (st != MMF_OK) return st;
+    if (!aligned16(x) || !aligned16(gamma) || !aligned16(packed) || !aligned16(scale) || !aligned16(y))
+        return MMF_ERR_MISALIGNED;
+    if (M == 0 || N == 0) return MMF_OK;
+    const size_t need = mmf_workspace_bytes(M, K, N);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return MMF_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return MMF_ERR_MISALIGNED;
+    DeviceState* dev;
+    if ((st = device_state(&dev)) != MMF_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    GemvPlan plan;
+    if (gemv_plan(static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), dev->num_sms, &plan)) {
+        GemvParams p{};
+        p.x = x;
+        p.gamma = gamma;
+        p.eps = eps;
+        p.packed = packed;
+        p.scale = scale;
+        p.y = y;
+        p.M = static_cast<int>(M);
+        p.K = static_cast<int>(K);
+        p.N = static_cast<int>(N);
+        p.rows_per_stage = plan.rows_per_stage;
+        p.rows_per_cta = plan.rows_per_cta;
+        p.stage_bytes = plan.stage_bytes;
+        return launch_gemv<true>(p, plan, s);
+    }
+    Workspace w = carve(workspace, M, K);
+    if ((st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s)) != MMF_OK) return st;
+    TcParams p{};
+    p.qsum = w.qsum;
+    p.absmax = w.absmax;
+    p.scale = scale;
+    p.y = y;
+    p.M = static_cast<int>(M);
+    p.K = static_cast<int>(K);
+    p.N = static_cast<int>(N);
+    return launch_tc(true, w.q, packed, p, s);
+}
+
+int mmf_hbm_copy(const void* src, void* dst, size_t bytes, void* stream) {
+    if (!src || !dst) return MMF_ERR_INVALID_ARG;
+    if ((bytes & 15u) != 0) return MMF_ERR_INVALID_ARG;
+    if (!aligned16(src) || !aligned16(dst)) return MMF_ERR_MISALIGNED;
+    if (bytes == 0) return MMF_OK;
+    DeviceState* dev;
+    mmf_status st = device_state(&dev);
+    if (st != MMF_OK) return st;
+    const int64_t n16 = static_cast<int64_t>(bytes / 16);
+    int64_t grid = (n16 + kCopyThreads - 1) / kCopyThreads;
+    if (grid > int64_t(dev->num_sms) * 4) grid = int64_t(dev->num_sms) * 4;
+    hbm_copy_kernel<<<static_cast<unsigned>(grid), kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16);
+    return launch_status();
+}
+
+int mmf_selftest_timeout(uint64_t limit_ns, int32_t* waited_out, void* stream) {
+    if (limit_ns == 0 || limit_ns > kWaitLimitNs) return MMF_ERR_INVALID_ARG;
+    if (waited_out && (reinterpret_cast<uintptr_t>(waited_out) & 3u)) return MMF_ERR_MISALIGNED;
+    DeviceState* dev;
+    mmf_status st = device_state(&dev);
+    if (st != MMF_OK) return st;
+    selftest_timeout_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, waited_out);
+    return launch_status();
+}
+
+int mmf_check_async(void* stream) {
+    DeviceState* dev;
+    mmf_status st = device_state(&dev);
+    if (st != MMF_OK) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MMF_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, mmf::g_error_word, sizeof(word)) != cudaSuccess) return MMF_ERR_CUDA;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(mmf::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return MMF_ERR_CUDA;
+        return MMF_ERR_TIMEOUT;
+    }
+    return MMF_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,183 @@
+"""ctypes binding of libmmf.so (the C ABI in include/mmf.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory and streams.  If the library has not
+been built this module raises on first use; there is no fallback path.
+
+Raw entry points (``lib()``) take integer device pointers; the tensor helpers
+below check dtypes/devices, allocate outputs with torch when none are given,
+and pass the current torch stream.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmmf.so")
+
+MMF_OK = 0
+STATUS = {
+    0: "MMF_OK", 1: "MMF_ERR_INVALID_ARG", 2: "MMF_ERR_UNSUPPORTED_SHAPE", 3: "MMF_ERR_MISALIGNED",
+    4: "MMF_ERR_WORKSPACE", 5: "MMF_ERR_CUDA", 6: "MMF_ERR_TIMEOUT", 7: "MMF_ERR_NO_DEVICE",
+}
+
+_lock = threading.Lock()
+_lib = None
+
+_P, _I64, _F, _SZ, _INT = C.c_void_p, C.c_int64, C.c_float, C.c_size_t, C.c_int
+
+# name -> (restype, argtypes); mirrors include/mmf.h
+SIGNATURES = {
+    "mmf_status_string": (C.c_char_p, [_INT]),
+    "mmf_version": (C.c_char_p, []),
+    "mmf_packed_bytes": (_SZ, [_I64, _I64]),
+    "mmf_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "mmf_pack_ternary": (_INT, [_P, _I64, _I64, _F, _P, _P, _P]),
+    "mmf_quantize_act": (_INT, [_P, _P, _F, _I64, _I64, _P, _P, _P]),
+    "mmf_ternary_acc": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "mmf_bitlinear_fwd": (_INT, [_P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "mmf_hbm_copy": (_INT, [_P, _P, _SZ, _P]),
+    "mmf_selftest_timeout": (_INT, [C.c_uint64, _P, _P]),
+    "mmf_check_async": (_INT, [_P]),
+}
+
+
+class MMFError(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+def lib() -> C.CDLL:
+    """Loads libmmf.so (once); raises if it is missing."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m bitlinear_rmsnorm_quant_b200.build`")
+            L = C.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                f = getattr(L, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = L
+    return _lib
+
+
+def check(status: int, what: str) -> None:
+    if status != MMF_OK:
+        raise MMFError(what, status)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# -- sizes ----------------------------------------------------------------------
+
+def packed_bytes(N: int, K: int) -> int:
+    return int(lib().mmf_packed_bytes(N, K))
+
+
+def workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().mmf_workspace_bytes(M, K, N))
+
+
+def version() -> str:
+    return lib().mmf_version().decode()
+
+
+# -- entry points ---------------------------------------------------------------
+
+def pack_ternary(W: torch.Tensor, eps_w: float = 1e-5, packed: torch.Tensor | None = None,
+                 scale: torch.Tensor | None = None, stream=None):
+    """fp32 W[N, K] -> (packed int32[N, K/16] holding uint32 words, scale fp32[1])."""
+    _dev(W, torch.float32, "W")
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty((N, K // 16), dtype=torch.int32, device=W.device)
+    if scale is None:
+        scale = torch.empty(4, dtype=torch.float32, device=W.device)[:1]
+    check(lib().mmf_pack_ternary(W.data_ptr(), N, K, eps_w, packed.data_ptr(), scale.data_ptr(), _stream(stream)),
+          "mmf_pack_ternary")
+    return packed, scale
+
+
+def quantize_act(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6, stream=None):
+    """bf16 x[M, K] -> (q int8[M, K], absmax fp32[M])."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(gamma, torch.float32, "gamma")
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    a = torch.empty(max(M, 4), dtype=torch.float32, device=x.device)[:M]
+    check(lib().mmf_quantize_act(x.data_ptr(), gamma.data_ptr(), eps, M, K, q.data_ptr(), a.data_ptr(),
+                                 _stream(stream)), "mmf_quantize_act")
+    return q, a
+
+
+def _workspace(M, K, N, device, workspace):
+    need = workspace_bytes(M, K, N)
+    if need == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    if workspace.numel() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    return workspace, workspace.numel()
+
+
+def ternary_acc(q: torch.Tensor, packed: torch.Tensor, N: int, workspace=None, out=None, stream=None):
+    """int8 q[M, K] x packed[N, K/16] -> int32 acc[M, N]."""
+    _dev(q, torch.int8, "q")
+    M, K = q.shape
+    acc = out if out is not None else torch.empty((M, N), dtype=torch.int32, device=q.device)
+    ws, ws_n = _workspace(M, K, N, q.device, workspace)
+    check(lib().mmf_ternary_acc(q.data_ptr(), packed.data_ptr(), M, K, N, acc.data_ptr(),
+                                ws.data_ptr() if ws is not None else None, ws_n, _stream(stream)),
+          "mmf_ternary_acc")
+    return acc
+
+
+def bitlinear_fwd(x: torch.Tensor, gamma: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, N: int,
+                  eps: float = 1e-6, workspace=None, out=None, stream=None):
+    """bf16 x[M, K] -> bf16 y[M, N]."""
+    _dev(x, torch.bfloat16, "x")
+    M, K = x.shape
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws, ws_n = _workspace(M, K, N, x.device, workspace)
+    check(lib().mmf_bitlinear_fwd(x.data_ptr(), gamma.data_ptr(), eps, packed.data_ptr(), scale.data_ptr(), M, K, N,
+                                  y.data_ptr(), ws.data_ptr() if ws is not None else None, ws_n, _stream(stream)),
+          "mmf_bitlinear_fwd")
+    return y
+
+
+def hbm_copy(src: torch.Tensor, dst: torch.Tensor, stream=None):
+    nbytes = src.numel() * src.element_size()
+    check(lib().mmf_hbm_copy(src.data_ptr(), dst.data_ptr(), nbytes, _stream(stream)), "mmf_hbm_copy")
+
+
+def selftest_timeout(limit_ns: int, waited_out: torch.Tensor | None = None, stream=None):
+    check(lib().mmf_selftest_timeout(limit_ns, waited_out.data_ptr() if waited_out is not None else None,
+                                     _stream(stream)), "mmf_selftest_timeout")
+
+
+def check_async(stream=None):
+    check(lib().mmf_check_async(_stream(stream)), "mmf_check_async")

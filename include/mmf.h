@@ -1,0 +1,174 @@
+/*
+ * mmf.h -- C ABI of the fused RMSNorm + BitLinear library for NVIDIA B200
+ * (sm_100a).  Library: bitlinear_rmsnorm_quant_b200/libmmf.so.
+ *
+ * The layer is the BitLinear dense layer of the MatMul-free language model
+ * ("Scalable MatMul-free Language Modeling", Zhu et al.):
+ *   - weights are ternary {-1, 0, +1}, obtained from full-precision latent
+ *     weights by absmean quantisation (datacamp.com, section "Thay MatMul bằng
+ *     các phép toán tam phân"; jiqizhixin.com, section "具有三值权重的
+ *     MatMul-free 密集层"), so the product needs only additions and
+ *     subtractions (ld246.com, section "三值权重的应用");
+ *   - the activations pass through RMSNorm before quantisation (datacamp.com,
+ *     component figure, item "RMS norm"), and RMSNorm and quantisation are one
+ *     fused operation that reads x from HBM once (ld246.com, section "融合
+ *     BitLinear 层的创新"; jiqizhixin.com, Algorithm 1);
+ *   - activations are quantised per token to int8 by absmax, accumulated in
+ *     int32, and rescaled by (absmax/127) * mean|W|.  The pages give no
+ *     formula; these are the plain definitions, stated per function below.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers owned by the caller unless stated.  The
+ *     library never allocates, frees or caches device memory and keeps no
+ *     pointer after a call returns.
+ *   - Every pointer must be 16-byte aligned (TMA and 128-bit loads).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous and ordered on that stream; results
+ *     are ready when the stream has reached the call.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Shapes: M tokens (0 <= M < 2^31), K = d_in (128 <= K <= 65536,
+ *     K % 128 == 0), N = d_out (0 <= N < 2^31).  M == 0 or N == 0 is a no-op
+ *     returning MMF_OK.
+ *   - Argument errors return synchronously and launch nothing.  A failed
+ *     launch returns MMF_ERR_CUDA.  A device-side wait that timed out (every
+ *     wait inside the kernels is bounded, about one second) is recorded in a
+ *     device error word, and the kernel that gave up returns without writing
+ *     its outputs; mmf_check_async reports (MMF_ERR_TIMEOUT) and clears it.
+ *   - The first call on a device does a one-time set-up (device properties,
+ *     kernel attributes, the driver's tensor-map entry point); make that
+ *     first call outside any CUDA graph capture.
+ *   - Entry points are thread-safe; calls that overlap on the GPU must not
+ *     write the same output or workspace buffer.
+ */
+#ifndef MMF_H
+#define MMF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mmf_status {
+    MMF_OK = 0,
+    MMF_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad eps */
+    MMF_ERR_UNSUPPORTED_SHAPE = 2, /* K not a multiple of 128 in [128, 65536], or too large */
+    MMF_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+    MMF_ERR_WORKSPACE = 4,         /* workspace missing or smaller than mmf_workspace_bytes */
+    MMF_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
+    MMF_ERR_TIMEOUT = 6,           /* a bounded device-side wait ran out */
+    MMF_ERR_NO_DEVICE = 7          /* no sm_100 device is current */
+} mmf_status;
+
+/* Human-readable name of a status code; never NULL. */
+const char* mmf_status_string(int status);
+
+/* Library version string, e.g. "mmf 0.1.0 sm_100a". */
+const char* mmf_version(void);
+
+/* Bytes of the packed ternary matrix for an N x K weight: N * K / 4. */
+size_t mmf_packed_bytes(int64_t N, int64_t K);
+
+/* Bytes of device workspace mmf_bitlinear_fwd and mmf_ternary_acc need for
+ * this shape; 0 when the shape takes the fused decode path (small M), which
+ * needs none.  Depends only on (M, K, N). */
+size_t mmf_workspace_bytes(int64_t M, int64_t K, int64_t N);
+
+/*
+ * mmf_pack_ternary -- absmean ternarisation and 2-bit packing of a latent
+ * weight matrix (datacamp.com, "Thay MatMul bằng các phép toán tam phân": the
+ * full-precision weights are scaled by their mean absolute value and rounded
+ * to the nearest of -1, 0, +1; read as a division, since a product would round
+ * every weight of a N(0, 0.02) matrix to 0).
+ *
+ *   beta   = mean over all N*K of |W|, summed in fp64 in a fixed order and
+ *            rounded once to fp32; written to scale[0].
+ *   w~     = clamp(rint(W / (beta + eps_w)), -1, 1), the division in fp32
+ *            (IEEE, round to nearest even), rint ties to even.
+ *   packed = uint32 [N][K/16], row-major, row pitch K/4 bytes.  Word j of row n
+ *            holds weights k = 16j + i, i = 0..15; weight i occupies bits
+ *            [8*(i%4) + 2*(i/4), +2) and stores the code w~ + 1
+ *            (0 = -1, 1 = 0, 2 = +1; 3 is never written).
+ *
+ * W: fp32 [N][K] row-major (nn.Linear layout, y = x W~^T).  eps_w >= 0.
+ * `packed` is also used as scratch before it receives the codes, so it must
+ * not alias W.  Deterministic: the same W gives the same bits on every run.
+ */
+int mmf_pack_ternary(const float* W, int64_t N, int64_t K, float eps_w,
+                     uint32_t* packed, float* scale, void* stream);
+
+/*
+ * mmf_quantize_act -- RMSNorm followed by per-token absmax int8 quantisation,
+ * one fused pass over x (the same arithmetic as inside mmf_bitlinear_fwd):
+ *   ms     = (float)(sum_k x_k^2 / K)      sum and quotient in fp64
+ *   inv    = 1 / sqrt(ms + eps)            fp32, correctly rounded
+ *   r_k    = (x_k * inv) * gamma_k         fp32, two roundings in this order
+ *   absmax = max(max_k |r_k|, 1e-5)        written to absmax[m]
+ *   q_k    = clamp(rint(r_k * (127/absmax)), -127, 127)
+ * x: bf16 [M][K]; gamma: fp32 [K]; q: int8 [M][K]; absmax: fp32 [M].
+ * eps >= 0.  x and q must not alias.
+ */
+int mmf_quantize_act(const uint16_t* x, const float* gamma, float eps,
+                     int64_t M, int64_t K, int8_t* q, float* absmax, void* stream);
+
+/*
+ * mmf_ternary_acc -- the ternary contraction alone, for parity checks:
+ *   acc[m][n] = sum over k with w~[n][k] = +1 of q[m][k]
+ *             - sum over k with w~[n][k] = -1 of q[m][k]      (int32, exact)
+ * q: int8 [M][K] (values in [-127, 127]); packed as from mmf_pack_ternary;
+ * acc: int32 [M][N].  Takes the same kernel path mmf_bitlinear_fwd takes for
+ * this (M, K, N), so it needs the same workspace.
+ */
+int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M,
+                    int64_t K, int64_t N, int32_t* acc, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
+ * mmf_bitlinear_fwd -- the fused BitLinear forward:
+ *   (q, absmax) = RMSNorm + quantisation of x, as in mmf_quantize_act
+ *   acc         = ternary contraction of q with the packed weights
+ *   y[m][n]     = bf16_rn((float)acc[m][n] * ((absmax[m] / 127) * scale[0]))
+ * x: bf16 [M][K]; gamma: fp32 [K]; packed/scale as from mmf_pack_ternary;
+ * y: bf16 [M][N].  workspace: device buffer of at least
+ * mmf_workspace_bytes(M, K, N) bytes (may be NULL when that is 0); it holds
+ * the int8 codes between the two kernels of the large-M path.  x, y and the
+ * workspace must not overlap.
+ */
+int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps,
+                      const uint32_t* packed, const float* scale, int64_t M,
+                      int64_t K, int64_t N, uint16_t* y, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
+ * mmf_hbm_copy -- streaming device-to-device copy of `bytes` bytes (a multiple
+ * of 16) with 128-bit loads and stores.  Measurement kernel: it gives the HBM
+ * bandwidth the roofline fractions are stated against.  src and dst must not
+ * overlap.
+ */
+int mmf_hbm_copy(const void* src, void* dst, size_t bytes, void* stream);
+
+/*
+ * mmf_selftest_timeout -- failure-detection self-test (no counterpart on the
+ * pages).  Launches one thread that waits on a shared-memory barrier nothing
+ * arrives at, with the same bounded wait the kernels use but a limit of
+ * limit_ns (0 < limit_ns <= 1e9).  The wait gives up, records a timeout in the
+ * device error word (so the next mmf_check_async returns MMF_ERR_TIMEOUT),
+ * writes 1 to *waited_out if waited_out is not NULL (device pointer, 4-byte
+ * aligned), and the kernel returns.  Nothing hangs or faults.
+ */
+int mmf_selftest_timeout(uint64_t limit_ns, int32_t* waited_out, void* stream);
+
+/*
+ * mmf_check_async -- synchronises `stream`, then reads and clears the device
+ * error word of the current device.  Returns MMF_ERR_TIMEOUT if a bounded
+ * wait in any earlier kernel ran out, MMF_ERR_CUDA if the stream reports an
+ * error, else MMF_OK.
+ */
+int mmf_check_async(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MMF_H */

@@ -1,0 +1,115 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every symbol
+include/mmf.h declares, and its host-side logic (sizes, status strings,
+argument checks that return before any CUDA call) behaves as documented."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mmf.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bitlinear_rmsnorm_quant_b200 import build, mmf
+    build.build()
+    return mmf.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mmf_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("mmf_pack_ternary", "mmf_bitlinear_fwd", "mmf_quantize_act", "mmf_ternary_acc",
+                 "mmf_check_async", "mmf_workspace_bytes", "mmf_packed_bytes"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    from bitlinear_rmsnorm_quant_b200 import mmf
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} not exported"
+        assert name in mmf.SIGNATURES, f"{name} not bound"
+
+
+def test_library_is_sm100a_only():
+    from bitlinear_rmsnorm_quant_b200 import build
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.NVCC_FLAGS)
+
+
+def test_sizes(L):
+    assert L.mmf_packed_bytes(2560, 6912) == 2560 * 6912 // 4
+    assert L.mmf_packed_bytes(-1, 128) == 0
+    # small M takes the fused decode kernel: no workspace
+    assert L.mmf_workspace_bytes(1, 2560, 2560) == 0
+    assert L.mmf_workspace_bytes(8, 6912, 2560) == 0
+    # large M: int8 codes + absmax + qsum, each 256-byte aligned
+    M, K = 8192, 2048
+    assert L.mmf_workspace_bytes(M, K, 5632) == M * K + 2 * ((4 * M + 255) // 256 * 256)
+    assert L.mmf_workspace_bytes(9, 256, 100) >= 9 * 256
+    # unsupported K
+    assert L.mmf_workspace_bytes(100, 100, 100) == 0
+
+
+def test_status_strings(L):
+    from bitlinear_rmsnorm_quant_b200 import mmf
+    for code, name in mmf.STATUS.items():
+        assert L.mmf_status_string(code).decode() == name
+    assert L.mmf_status_string(99).decode() == "MMF_ERR_UNKNOWN"
+    assert L.mmf_version().decode().startswith("mmf ")
+
+
+# Fake, never-dereferenced device addresses: the checks below return before
+# the library touches CUDA.
+A = 0x10000
+MIS = 0x10008
+
+
+def test_argument_errors_need_no_device(L):
+    # null pointers
+    assert L.mmf_pack_ternary(None, 16, 128, 1e-5, A, A, None) == 1
+    assert L.mmf_bitlinear_fwd(A, A, 1e-6, None, A, 1, 128, 16, A, None, 0, None) == 1
+    assert L.mmf_quantize_act(A, None, 1e-6, 1, 128, A, A, None) == 1
+    assert L.mmf_ternary_acc(A, A, 1, 128, 16, None, None, 0, None) == 1
+    # bad eps
+    assert L.mmf_pack_ternary(A, 16, 128, -1.0, A, A, None) == 1
+    assert L.mmf_quantize_act(A, A, float("nan"), 1, 128, A, A, None) == 1
+    # K not a positive multiple of 128, or above the limit
+    for K in (0, 64, 100, 130, 65536 + 128):
+        assert L.mmf_bitlinear_fwd(A, A, 1e-6, A, A, 1, K, 16, A, None, 0, None) == 2
+    # negative sizes
+    assert L.mmf_bitlinear_fwd(A, A, 1e-6, A, A, -1, 128, 16, A, None, 0, None) == 1
+    # misaligned pointers
+    assert L.mmf_bitlinear_fwd(MIS, A, 1e-6, A, A, 1, 128, 16, A, None, 0, None) == 3
+    assert L.mmf_pack_ternary(A, 16, 128, 1e-5, MIS, A, None) == 3
+    assert L.mmf_hbm_copy(A, MIS, 64, None) == 3
+    assert L.mmf_hbm_copy(A, A, 15, None) == 1
+    # missing or short workspace on the large-M path
+    assert L.mmf_bitlinear_fwd(A, A, 1e-6, A, A, 4096, 2048, 2048, A, None, 0, None) == 4
+    assert L.mmf_bitlinear_fwd(A, A, 1e-6, A, A, 4096, 2048, 2048, A, A, 1024, None) == 4
+    assert L.mmf_ternary_acc(A, A, 4096, 2048, 2048, A, None, 0, None) == 4
+    # empty problems are no-ops that launch nothing
+    assert L.mmf_bitlinear_fwd(A, A, 1e-6, A, A, 0, 128, 16, A, None, 0, None) == 0
+    assert L.mmf_bitlinear_fwd(A, A, 1e-6, A, A, 3, 128, 0, A, None, 0, None) == 0
+    assert L.mmf_pack_ternary(A, 0, 128, 1e-5, A, A, None) == 0
+    assert L.mmf_hbm_copy(A, A, 0, None) == 0
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device path")
+def test_no_device_is_reported(L):
+    assert L.mmf_bitlinear_fwd(A, A, 1e-6, A, A, 1, 128, 16, A, None, 0, None) == 7
+    assert L.mmf_check_async(None) == 7
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    from bitlinear_rmsnorm_quant_b200 import mmf
+    monkeypatch.setattr(mmf, "_lib", None)
+    monkeypatch.setattr(mmf, "LIB_PATH", "/nonexistent/libmmf.so")
+    with pytest.raises(RuntimeError, match="missing"):
+        mmf.lib()

@@ -1,0 +1,284 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bars: packed words, beta and int32 accumulators bit-exact; y within max
+relative error 1e-2 (floored, see gpu_cases); at most 0.1% of int8 activation
+codes differ, and then by one.  Sizes span several tiles with ragged tails on
+both kernel paths (fused decode GEMV for M <= 8, tcgen05 GEMM above), and the
+full configuration sizes are checked on sampled tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bitlinear_rmsnorm_quant_b200 import mmf
+from bitlinear_rmsnorm_quant_b200 import workloads as WL
+from gpu_cases import (Q_MAX_DIFF_FRAC, Y_REL_TOL, bits_np, make_layer, q_diff_stats, y_rel_error)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+EPS = 1e-6
+EPS_W = 1e-5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from bitlinear_rmsnorm_quant_b200 import build
+    build.build()
+    torch.cuda.set_device(0)
+    yield
+    mmf.check_async()
+
+
+def _pack(W):
+    packed, scale = mmf.pack_ternary(W.to(DEV), EPS_W)
+    return packed, scale
+
+
+def _oracle_codes(oracle, W):
+    wt, beta = oracle.absmean_ternary(W.numpy(), EPS_W)
+    return wt, beta
+
+
+# -- packer ------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K", [(256, 256), (1, 128), (3, 384), (1000, 1024), (2816, 1024), (2560, 6912),
+                                 (5632, 2048)])
+def test_pack_bit_exact(oracle, N, K):
+    _, _, W = make_layer(7, 1, K, N)
+    packed, scale = _pack(W)
+    torch.cuda.synchronize()
+    wt, beta = _oracle_codes(oracle, W)
+    assert np.float32(scale.item()) == beta
+    ref = oracle.encode_packed(wt)
+    got = packed.cpu().numpy().view(np.uint32)
+    assert np.array_equal(got, ref)
+
+
+def test_pack_deterministic():
+    _, _, W = make_layer(8, 1, 2560, 2560)
+    Wd = W.to(DEV)
+    p1, s1 = mmf.pack_ternary(Wd, EPS_W)
+    p2, s2 = mmf.pack_ternary(Wd, EPS_W)
+    torch.cuda.synchronize()
+    assert torch.equal(p1, p2) and torch.equal(s1, s2)
+
+
+def test_pack_special_matrices(oracle):
+    # W = c*I gives the identity; a constant matrix gives all +1
+    K = 256
+    W = torch.eye(K, dtype=torch.float32) * 0.75
+    packed, scale = _pack(W)
+    wt, bad = oracle.decode_packed(packed.cpu().numpy().view(np.uint32), K)
+    assert bad == 0 and np.array_equal(wt, np.eye(K, dtype=np.int8))
+    packed, _ = _pack(torch.full((16, K), -0.3))
+    wt, _ = oracle.decode_packed(packed.cpu().numpy().view(np.uint32), K)
+    assert (wt == -1).all()
+
+
+# -- RMSNorm + quantisation ------------------------------------------------------------
+
+@pytest.mark.parametrize("M,K,outliers", [(16, 256, 0.0), (5, 128, 0.0), (300, 2048, 0.0), (37, 6912, 0.01),
+                                          (64, 5632, 0.0)])
+def test_quantize_act(oracle, M, K, outliers):
+    x, g, _ = make_layer(9, M, K, 1, outlier_frac=outliers)
+    q, a = mmf.quantize_act(x.to(DEV), g.to(DEV), EPS)
+    torch.cuda.synchronize()
+    q_ref, a_ref = oracle.rmsnorm_quant(bits_np(x), g.numpy(), EPS)
+    frac, mx = q_diff_stats(q.cpu().numpy(), q_ref)
+    assert mx <= 1 and frac <= Q_MAX_DIFF_FRAC
+    assert np.allclose(a.cpu().numpy(), a_ref, rtol=2e-7, atol=0)
+
+
+def test_quantize_special_rows(oracle):
+    K = 512
+    x = torch.zeros(4, K, dtype=torch.bfloat16)
+    x[1] = 3.0
+    x[2] = -0.5
+    x[3, 7] = 1.0
+    g = torch.ones(K)
+    q, a = mmf.quantize_act(x.to(DEV), g.to(DEV), EPS)
+    torch.cuda.synchronize()
+    q = q.cpu()
+    assert (q[0] == 0).all() and a[0].item() == np.float32(1e-5)
+    assert (q[1] == 127).all() and (q[2] == -127).all()
+    assert q[3, 7] == 127 and (q[3].abs().sum() == 127)
+
+
+# -- ternary contraction: int32 bit-exact on the kernel's own q and packed W --------------
+
+ACC_SHAPES = [
+    # (M, K, N) decode GEMV path (M <= 8)
+    (1, 128, 1), (1, 256, 256), (2, 1024, 1000), (3, 2560, 333), (8, 6912, 2560), (5, 2816, 1024),
+    # tcgen05 path: several 128-row tiles, token tiles, K stages, ragged tails
+    (9, 256, 300), (16, 256, 256), (17, 384, 129), (32, 2560, 640), (100, 1024, 257), (256, 512, 384),
+    (300, 384, 300), (513, 2048, 200),
+]
+
+
+@pytest.mark.parametrize("M,K,N", ACC_SHAPES)
+def test_ternary_acc_bit_exact(oracle, M, K, N):
+    x, g, W = make_layer(10, M, K, N)
+    packed, _ = _pack(W)
+    q, _ = mmf.quantize_act(x.to(DEV), g.to(DEV), EPS)
+    acc = mmf.ternary_acc(q, packed, N)
+    torch.cuda.synchronize()
+    wt, bad = oracle.decode_packed(packed.cpu().numpy().view(np.uint32), K)
+    assert bad == 0
+    ref = oracle.ternary_acc(q.cpu().numpy(), wt)
+    got = acc.cpu().numpy()
+    assert np.array_equal(got, ref), f"{np.count_nonzero(got != ref)} of {got.size} differ"
+
+
+def test_ternary_acc_extreme_codes(oracle):
+    # every activation at +-127 and every weight at +-1: the largest |acc|
+    M, K, N = 20, 6912, 256
+    q = torch.full((M, K), 127, dtype=torch.int8)
+    q[1::2] = -127
+    W = torch.ones(N, K)
+    W[N // 2:] = -1.0
+    packed, _ = _pack(W)
+    acc = mmf.ternary_acc(q.to(DEV), packed, N)
+    acc1 = mmf.ternary_acc(q[:1].to(DEV), packed, N)
+    torch.cuda.synchronize()
+    wt, _ = oracle.decode_packed(packed.cpu().numpy().view(np.uint32), K)
+    assert np.array_equal(acc.cpu().numpy(), oracle.ternary_acc(q.numpy(), wt))
+    assert np.array_equal(acc1.cpu().numpy(), oracle.ternary_acc(q[:1].numpy(), wt))
+    assert abs(int(acc[0, 0])) == 127 * K
+
+
+# -- whole layer against the oracle ----------------------------------------------------------
+
+def _layer_parity(oracle, x, g, W, sample_tokens=None):
+    packed, scale = _pack(W)
+    y = mmf.bitlinear_fwd(x.to(DEV), g.to(DEV), packed, scale, W.shape[0], EPS)
+    torch.cuda.synchronize()
+    xs = x if sample_tokens is None else x[sample_tokens]
+    ys = y if sample_tokens is None else y[torch.as_tensor(sample_tokens, device=y.device)]
+    y_ref, beta = oracle.bitlinear(bits_np(xs), g.numpy(), EPS, W.numpy(), EPS_W)
+    assert np.float32(scale.item()) == beta
+    err = y_rel_error(bits_np(ys), y_ref)
+    assert err <= Y_REL_TOL, err
+    return err
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 128, 16), (1, 1024, 2816), (4, 2560, 1000), (8, 6912, 2560),
+                                   (9, 256, 256), (16, 256, 256), (33, 2048, 500), (300, 384, 300),
+                                   (1000, 1024, 384)])
+def test_bitlinear_parity(oracle, M, K, N):
+    x, g, W = make_layer(11, M, K, N)
+    _layer_parity(oracle, x, g, W)
+
+
+def test_smoke_config(oracle):
+    w = WL.SMOKE
+    p = w.projections[0]
+    x, g, W = make_layer(w.seed, w.M, p.K, p.N)
+    _layer_parity(oracle, x, g, W)
+
+
+@pytest.mark.parametrize("wl", [WL.DECODE_370M, WL.decode_2p7b(1), WL.decode_2p7b(8), WL.decode_2p7b(32)],
+                         ids=lambda w: w.name)
+def test_decode_configs(oracle, wl):
+    for j, p in enumerate(wl.projections):
+        x, g, W = make_layer(wl.seed, wl.M, p.K, p.N, index=p.input_index, outlier_frac=wl.outlier_frac)
+        _layer_parity(oracle, x, g, W)
+
+
+def test_prefill_config_sampled(oracle):
+    """Full prefill size (M=8192) on the GPU; the oracle checks 48 sampled tokens."""
+    wl = WL.PREFILL_1P3B
+    rng = np.random.default_rng(5)
+    for p in wl.projections:
+        x, g, W = make_layer(wl.seed, wl.M, p.K, p.N, index=p.input_index)
+        tokens = np.sort(rng.choice(wl.M, 48, replace=False))
+        _layer_parity(oracle, x, g, W, sample_tokens=tokens)
+
+
+def test_zero_and_degenerate_tokens(oracle):
+    K, N = 1024, 512
+    x, g, W = make_layer(12, 40, K, N)
+    x[3] = 0.0
+    x[7] = 2.5
+    x[11, :] = 0.0
+    x[11, 5] = -7.0
+    _layer_parity(oracle, x, g, W)
+    _layer_parity(oracle, x[:4], g, W)     # decode path with a zero token
+    packed, scale = _pack(W)
+    y = mmf.bitlinear_fwd(x.to(DEV), g.to(DEV), packed, scale, N, EPS)
+    torch.cuda.synchronize()
+    assert (y[3] == 0).all()
+
+
+def test_empty_problems():
+    K, N = 256, 64
+    x = torch.zeros(0, K, dtype=torch.bfloat16, device=DEV)
+    g = torch.ones(K, device=DEV)
+    W = torch.randn(N, K, device=DEV)
+    packed, scale = mmf.pack_ternary(W)
+    y = mmf.bitlinear_fwd(x, g, packed, scale, N)
+    assert y.shape == (0, N)
+    y = mmf.bitlinear_fwd(torch.zeros(3, K, dtype=torch.bfloat16, device=DEV), g, packed, scale, 0)
+    assert y.shape == (3, 0)
+    torch.cuda.synchronize()
+
+
+def test_fwd_deterministic():
+    for M in (1, 64):
+        x, g, W = make_layer(13, M, 2048, 1024)
+        packed, scale = _pack(W)
+        xd, gd = x.to(DEV), g.to(DEV)
+        y1 = mmf.bitlinear_fwd(xd, gd, packed, scale, 1024)
+        y2 = mmf.bitlinear_fwd(xd, gd, packed, scale, 1024)
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y2)
+
+
+# -- error paths on the device -----------------------------------------------------------------
+
+def test_argument_errors_on_device():
+    K, N = 256, 64
+    x = torch.zeros(64, K, dtype=torch.bfloat16, device=DEV)
+    g = torch.ones(K, device=DEV)
+    packed, scale = mmf.pack_ternary(torch.randn(N, K, device=DEV))
+    L = mmf.lib()
+    s = torch.cuda.current_stream().cuda_stream
+    y = torch.empty(64, N, dtype=torch.bfloat16, device=DEV)
+    need = mmf.workspace_bytes(64, K, N)
+    assert need > 0
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    assert L.mmf_bitlinear_fwd(x.data_ptr(), g.data_ptr(), 1e-6, packed.data_ptr(), scale.data_ptr(), 64, K, N,
+                               y.data_ptr(), ws.data_ptr(), need - 1, s) == 4
+    assert L.mmf_bitlinear_fwd(x.data_ptr() + 2, g.data_ptr(), 1e-6, packed.data_ptr(), scale.data_ptr(), 64, K, N,
+                               y.data_ptr(), ws.data_ptr(), need, s) == 3
+    assert L.mmf_bitlinear_fwd(x.data_ptr(), g.data_ptr(), 1e-6, packed.data_ptr(), scale.data_ptr(), 64, 200, N,
+                               y.data_ptr(), ws.data_ptr(), need, s) == 2
+    assert L.mmf_bitlinear_fwd(x.data_ptr(), g.data_ptr(), 1e-6, packed.data_ptr(), scale.data_ptr(), 64, K, N,
+                               y.data_ptr(), ws.data_ptr(), need, s) == 0
+    mmf.check_async()
+
+
+def test_timeout_is_reported_not_hung():
+    """A bounded wait on a barrier nothing arrives at gives up, is reported by
+    mmf_check_async as MMF_ERR_TIMEOUT, and leaves the context usable."""
+    mmf.check_async()
+    flag = torch.zeros(4, dtype=torch.int32, device=DEV)
+    mmf.selftest_timeout(20_000_000, flag)  # 20 ms
+    with pytest.raises(mmf.MMFError) as e:
+        mmf.check_async()
+    assert e.value.status == 6
+    assert int(flag[0]) == 1
+    mmf.check_async()                        # cleared
+    a = torch.arange(1024, dtype=torch.float32, device=DEV)
+    b = torch.empty_like(a)
+    mmf.hbm_copy(a, b)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_hbm_copy():
+    a = torch.randint(0, 1 << 30, (1 << 22,), dtype=torch.int32, device=DEV)
+    b = torch.empty_like(a)
+    mmf.hbm_copy(a, b)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
