@@ -48,8 +48,8 @@ cudaError_t set_tc_attrs() {
 
 template <int MT>
 cudaError_t set_gemv_attrs() {
-    cudaError_t e = set_smem(gemv_kernel<MT, true>, 200 * 1024);
-    if (e == cudaSuccess) e = set_smem(gemv_kernel<MT, false>, 200 * 1024);
+    cudaError_t e = set_smem(gemv_kernel<MT, true>, kGemvSmemBudget);
+    if (e == cudaSuccess) e = set_smem(gemv_kernel<MT, false>, kGemvSmemBudget);
     return e;
 }
 
@@ -248,12 +248,12 @@ size_t mmf_workspace_bytes(int64_t M, int64_t K, int64_t N) {
 
 int mmf_pack_ternary(const float* W, int64_t N, int64_t K, float eps_w, uint32_t* packed, float* scale,
                      void* stream) {
-    if (!W || !packed || !scale) return MMF_ERR_INVALID_ARG;
     if (!(eps_w >= 0.0f) || eps_w > 1e30f) return MMF_ERR_INVALID_ARG;
     mmf_status st = check_shape(0, K, N);
     if (st != MMF_OK) return st;
+    if (N == 0) return MMF_OK;  // empty: pointers may be NULL, nothing is written
+    if (!W || !packed || !scale) return MMF_ERR_INVALID_ARG;
     if (!aligned16(W) || !aligned16(packed) || !aligned16(scale)) return MMF_ERR_MISALIGNED;
-    if (N == 0) return MMF_OK;
     DeviceState* dev;
     if ((st = device_state(&dev)) != MMF_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -275,12 +275,12 @@ int mmf_pack_ternary(const float* W, int64_t N, int64_t K, float eps_w, uint32_t
 
 int mmf_quantize_act(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K, int8_t* q,
                      float* absmax, void* stream) {
-    if (!x || !gamma || !q || !absmax) return MMF_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || eps > 1e30f) return MMF_ERR_INVALID_ARG;
     mmf_status st = check_shape(M, K, 1);
     if (st != MMF_OK) return st;
-    if (!aligned16(x) || !aligned16(gamma) || !aligned16(q) || !aligned16(absmax)) return MMF_ERR_MISALIGNED;
     if (M == 0) return MMF_OK;
+    if (!x || !gamma || !q || !absmax) return MMF_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gamma) || !aligned16(q) || !aligned16(absmax)) return MMF_ERR_MISALIGNED;
     DeviceState* dev;
     if ((st = device_state(&dev)) != MMF_OK) return st;
     return launch_quant(x, gamma, eps, M, K, q, absmax, nullptr, static_cast<cudaStream_t>(stream));
@@ -288,11 +288,11 @@ int mmf_quantize_act(const uint16_t* x, const float* gamma, float eps, int64_t M
 
 int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t K, int64_t N, int32_t* acc,
                     void* workspace, size_t workspace_bytes, void* stream) {
-    if (!q || !packed || !acc) return MMF_ERR_INVALID_ARG;
     mmf_status st = check_shape(M, K, N);
     if (st != MMF_OK) return st;
-    if (!aligned16(q) || !aligned16(packed) || !aligned16(acc)) return MMF_ERR_MISALIGNED;
     if (M == 0 || N == 0) return MMF_OK;
+    if (!q || !packed || !acc) return MMF_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(packed) || !aligned16(acc)) return MMF_ERR_MISALIGNED;
     const size_t need = mmf_workspace_bytes(M, K, N);
     if (need > 0 && (!workspace || workspace_bytes < need)) return MMF_ERR_WORKSPACE;
     if (workspace && !aligned16(workspace)) return MMF_ERR_MISALIGNED;
@@ -311,6 +311,7 @@ int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t 
         p.rows_per_stage = plan.rows_per_stage;
         p.rows_per_cta = plan.rows_per_cta;
         p.stage_bytes = plan.stage_bytes;
+        p.stages = plan.stages;
         return launch_gemv<false>(p, plan, s);
     }
     Workspace w = carve(workspace, M, K);
@@ -328,13 +329,13 @@ int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t 
 int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps, const uint32_t* packed, const float* scale,
                       int64_t M, int64_t K, int64_t N, uint16_t* y, void* workspace, size_t workspace_bytes,
                       void* stream) {
-    if (!x || !gamma || !packed || !scale || !y) return MMF_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || eps > 1e30f) return MMF_ERR_INVALID_ARG;
     mmf_status st = check_shape(M, K, N);
     if (st != MMF_OK) return st;
+    if (M == 0 || N == 0) return MMF_OK;
+    if (!x || !gamma || !packed || !scale || !y) return MMF_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(gamma) || !aligned16(packed) || !aligned16(scale) || !aligned16(y))
         return MMF_ERR_MISALIGNED;
-    if (M == 0 || N == 0) return MMF_OK;
     const size_t need = mmf_workspace_bytes(M, K, N);
     if (need > 0 && (!workspace || workspace_bytes < need)) return MMF_ERR_WORKSPACE;
     if (workspace && !aligned16(workspace)) return MMF_ERR_MISALIGNED;
@@ -356,6 +357,7 @@ int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps, const ui
         p.rows_per_stage = plan.rows_per_stage;
         p.rows_per_cta = plan.rows_per_cta;
         p.stage_bytes = plan.stage_bytes;
+        p.stages = plan.stages;
         return launch_gemv<true>(p, plan, s);
     }
     Workspace w = carve(workspace, M, K);

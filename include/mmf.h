@@ -28,7 +28,8 @@
  *   - bf16 tensors are passed as uint16_t bit patterns.
  *   - Shapes: M tokens (0 <= M < 2^31), K = d_in (128 <= K <= 65536,
  *     K % 128 == 0), N = d_out (0 <= N < 2^31).  M == 0 or N == 0 is a no-op
- *     returning MMF_OK.
+ *     returning MMF_OK once the scalar arguments and K are valid; the buffer
+ *     pointers of an empty problem are not checked and may be NULL.
  *   - Argument errors return synchronously and launch nothing.  A failed
  *     launch returns MMF_ERR_CUDA.  A device-side wait that timed out (every
  *     wait inside the kernels is bounded, about one second) is recorded in a
