@@ -227,25 +227,47 @@ def run_ours(args, dist: Dist):
     ws = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=dev)
     lib = mmf.lib()
 
-    calls = []
+    # one call per (layer set, shared input): the token mixer's 4 projections,
+    # the channel mixer's gate/up pair and the down projection each share x
+    flags = 0 if args.no_pdl else mmf.FWD_PDL
+    calls = []          # (function, args without the stream)
+    keep = []           # ctypes arrays that must outlive the graph
     launches_per_step = 0
     bytes_per_step = 0
     ops_per_step = 0
     for l in range(L):
+        groups = {}
         for j, p in enumerate(wl.projections):
-            x, g = xs[l, p.input_index], gs[l, p.input_index]
-            calls.append((x.data_ptr(), g.data_ptr(), wl.eps, packed[l, j].data_ptr(), scales[l, j].data_ptr(),
-                          M, p.K, p.N, ys[l, j].data_ptr(), ws.data_ptr(), ws.numel()))
-            launches_per_step += 1 if mmf.workspace_bytes(M, p.K, p.N) == 0 else 2
-            bytes_per_step += proj_bytes(M, p.K, p.N)
-            ops_per_step += proj_ops(M, p.K, p.N)
+            groups.setdefault(p.input_index, []).append(j)
+        for idx, js in sorted(groups.items()):
+            K = wl.projections[js[0]].K
+            x, g = xs[l, idx], gs[l, idx]
+            if args.api == "group":
+                arr = mmf.projection_array([(packed[l, j], scales[l, j], ys[l, j], wl.projections[j].N) for j in js])
+                keep.append(arr)
+                calls.append((lib.mmf_bitlinear_fwd_group, (x.data_ptr(), g.data_ptr(), wl.eps, M, K, arr, len(js),
+                                                            ws.data_ptr(), ws.numel(), flags)))
+                tc = mmf.workspace_bytes(M, K, 1) > 0
+                launches_per_step += (1 + len(js)) if tc else 1
+            else:
+                for j in js:
+                    p = wl.projections[j]
+                    calls.append((lib.mmf_bitlinear_fwd, (x.data_ptr(), g.data_ptr(), wl.eps, packed[l, j].data_ptr(),
+                                                          scales[l, j].data_ptr(), M, p.K, p.N, ys[l, j].data_ptr(),
+                                                          ws.data_ptr(), ws.numel())))
+                    launches_per_step += 1 if mmf.workspace_bytes(M, p.K, p.N) == 0 else 2
+            for j in js:
+                p = wl.projections[j]
+                bytes_per_step += p.N * p.K // 4 + 2 * M * p.N + 4
+                ops_per_step += proj_ops(M, p.K, p.N)
+            bytes_per_step += 2 * M * K + 4 * K      # x and gamma once per shared input
     decode_path = all(mmf.workspace_bytes(M, p.K, p.N) == 0 for p in wl.projections)
 
     def step(stream_ptr):
-        for c in calls:
-            rc = lib.mmf_bitlinear_fwd(*c, stream_ptr)
+        for f, a in calls:
+            rc = f(*a, stream_ptr)
             if rc != 0:
-                raise mmf.MMFError("mmf_bitlinear_fwd", rc)
+                raise mmf.MMFError(f.__name__, rc)
 
     # first calls outside capture (one-time per-device set-up), then capture
     step(torch.cuda.current_stream().cuda_stream)
@@ -346,6 +368,8 @@ def run_ours(args, dist: Dist):
             "l2": "inputs larger than L2: packed weights of all layer sets exceed 126 MB"
                   if sum(p.N * p.K // 4 for p in wl.projections) * L > L2_BYTES else "working set below L2",
             "graph": "one CUDA graph per step", "parallelism": f"dp{dist.world} (token-parallel replicas)",
+            "api": "mmf_bitlinear_fwd_group" if args.api == "group" else "mmf_bitlinear_fwd",
+            "pdl": not args.no_pdl and args.api == "group", "launches_per_step": launches_per_step,
         },
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s (one token through one BitLinear layer set)",
@@ -453,6 +477,9 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--layers", type=int, default=0, help="layer sets per step (default per workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--api", choices=("group", "single"), default="group",
+                    help="group: one call per set of projections sharing x; single: one call per projection")
+    ap.add_argument("--no-pdl", action="store_true", help="plain stream-ordered launches")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

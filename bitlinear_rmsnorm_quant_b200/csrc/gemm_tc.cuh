@@ -94,6 +94,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_alloc(&tmem_base_s, L::tmem_cols);
         tmem_relinquish();
     }
+    // the codes, sums and scales come from the kernel before (no-op unless
+    // launched as a programmatic dependent)
+    pdl_wait();
+    pdl_launch_dependents();
     if (warp >= 4) {
         // per-token epilogue constants of this tile
         for (int i = threadIdx.x - 128; i < BT; i += 128) {

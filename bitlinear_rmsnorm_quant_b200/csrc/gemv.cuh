@@ -1,6 +1,8 @@
 // gemv.cuh -- decode-regime fused BitLinear (small M): RMSNorm + int8
-// quantisation of the M tokens into shared memory, then the ternary
-// contraction over a stream of 2-bit packed weights on CUDA cores.
+// quantisation of the M tokens in shared memory, then the ternary contraction
+// over a stream of 2-bit packed weights on CUDA cores.  One launch serves a
+// group of up to kGemvMaxProj projections that share the input x (the token
+// mixer's gate projections, the channel mixer's gate/up pair).
 //
 // The contraction follows the pages' ternary rule (ld246.com, section
 // "三值权重的应用": +1 adds the input, -1 subtracts it, 0 skips it).  The
@@ -13,13 +15,16 @@
 // power-of-four lanes are shifted back and summed once per row, and the
 // per-token sum_k q_k is subtracted once.  All integer, exact.
 //
-// CTA: 8 compute warps + 1 producer warp.  The CTA owns a contiguous range of
-// output rows; the producer first bulk-copies (TMA) the M rows of x into shared
-// memory, then streams the CTA's weight rows (contiguous in memory) into a ring
-// of shared-memory stages, so the weight fetch overlaps the normalisation.  Compute
-// warps take groups of 4 rows; 8 lanes cover one row, lane l reading 16-byte
-// chunks l, l+8, ... (64 weights each); a row's 8 partials meet in a 3-step
-// warp-shuffle tree.
+// CTA: 8 compute warps + 1 producer warp.  The group's weight rows form one
+// concatenated row space; each CTA owns a contiguous range of it.  The
+// producer bulk-copies (TMA) the CTA's weight rows into a ring of small
+// shared-memory stages and gamma into shared memory, then waits for the
+// previous kernel on the stream (programmatic dependent launch; a no-op when
+// the launch is not programmatic), then copies the M rows of x.  So under PDL
+// the weight stream overlaps the previous kernel and only x waits for it.
+// Compute warps take groups of 4 rows; 8 lanes cover one row, lane l reading
+// 16-byte chunks l, l+8, ... (64 weights each); a row's 8 partials meet in a
+// 3-step warp-shuffle tree.
 #pragma once
 #include "common.cuh"
 
@@ -27,76 +32,98 @@ namespace mmf {
 
 constexpr int kGemvComputeWarps = 8;
 constexpr int kGemvThreads = (kGemvComputeWarps + 1) * 32;
-constexpr int kGemvStages = 4;
+constexpr int kGemvMaxStages = 8;
 constexpr int kGemvMaxTokens = 8;
-constexpr int kGemvStageTarget = 32768;  // bytes of packed weights per stage
-
-struct GemvParams {
-    const uint16_t* x;       // bf16 [M][K]      (fused mode)
-    const float* gamma;      // fp32 [K]         (fused mode)
-    const int8_t* q_in;      // int8 [M][K]      (contraction-only mode)
-    const uint32_t* packed;  // [N][K/16]
-    const float* scale;      // beta             (fused mode)
-    uint16_t* y;             // bf16 [M][N]      (fused mode)
-    int32_t* acc;            // int32 [M][N]     (contraction-only mode)
-    float eps;
-    int M, K, N;
-    int rows_per_stage;      // multiple of 4
-    int rows_per_cta;
-    int stage_bytes;         // rows_per_stage * K/4
-    int stages;              // 2 .. kGemvStages
-};
-
+constexpr int kGemvMaxProj = 8;
+constexpr int kGemvStageTarget = 8192;       // bytes of packed weights per stage
+constexpr int kGemvSmemTwoCta = 110 * 1024;  // two CTAs per SM fit under this
 constexpr int kGemvSmemBudget = 200 * 1024;
 
+struct GemvParams {
+    const uint16_t* x;                      // bf16 [M][K]      (fused mode)
+    const float* gamma;                     // fp32 [K]         (fused mode)
+    const int8_t* q_in;                     // int8 [M][K]      (contraction-only mode)
+    const uint32_t* packed[kGemvMaxProj];   // [N_g][K/16]
+    const float* scale[kGemvMaxProj];       // beta_g           (fused mode)
+    uint16_t* y[kGemvMaxProj];              // bf16 [M][N_g]    (fused mode)
+    int32_t* acc;                           // int32 [M][N]     (contraction-only mode, one projection)
+    int row_start[kGemvMaxProj + 1];        // prefix sums of N_g
+    float eps;
+    int M, K, nproj;
+    int rows_per_stage;                     // multiple of 4
+    int rows_per_cta;
+    int stage_bytes;                        // rows_per_stage * K/4
+    int stages;                             // 1 .. kGemvMaxStages
+};
+
 // Host-side shape of the launch; returns false if the shape does not fit.
-// Shared memory: `stages` weight stages, the M bf16 rows of x (3 bytes per
-// activation with their int8 codes).  The plan depends only on (M, K, N) and
-// the SM count; feasibility depends only on (M, K).
+// Shared memory holds `stages` weight stages and the activations: x (bf16),
+// its int8 codes and gamma (fp32).  Feasibility depends only on (M, K).
 struct GemvPlan {
     int rows_per_stage, stage_bytes, rows_per_cta, grid, stages;
     size_t smem_bytes;
 };
 
-inline bool gemv_plan(int M, int K, int N, int num_sms, GemvPlan* plan) {
-    if (M < 1 || M > kGemvMaxTokens) return false;
+inline size_t gemv_act_bytes(int M, int K) { return static_cast<size_t>(3) * M * K + static_cast<size_t>(4) * K; }
+
+inline bool gemv_plan(int M, int K, int64_t R, int num_sms, GemvPlan* plan) {
+    if (M < 1 || M > kGemvMaxTokens || R < 1) return false;
     const int rowbytes = K / 4;
-    const size_t act = static_cast<size_t>(3) * M * K;
+    const size_t act = gemv_act_bytes(M, K);
     int rs = 4 * (kGemvStageTarget / (4 * rowbytes));
+    if (rs < 4) rs = 4;
     if (rs > 64) rs = 64;
-    int st = kGemvStages;
-    for (;;) {
-        if (rs < 4) return false;
-        if (static_cast<size_t>(st) * rs * rowbytes + act <= static_cast<size_t>(kGemvSmemBudget)) break;
-        if (st > 2) --st;
-        else rs -= 4;
-    }
-    plan->rows_per_stage = rs;
-    plan->stage_bytes = rs * rowbytes;
-    plan->stages = st;
-    int grid = (N + 3) / 4;
+    int grid = static_cast<int>((R + 3) / 4);
     if (grid > num_sms) grid = num_sms;
-    if (grid < 1) grid = 1;
-    int per = (N + grid - 1) / grid;
+    int per = static_cast<int>((R + grid - 1) / grid);
     per = (per + 3) & ~3;
-    plan->rows_per_cta = per;
-    plan->grid = (N + per - 1) / per;
-    plan->smem_bytes = static_cast<size_t>(st) * plan->stage_bytes + act;
-    return true;
+    const int want = (per + rs - 1) / rs;  // stages that hold the CTA's whole slab
+    // Prefer a ring that holds the whole slab within the two-CTA budget, then
+    // fewer stages, then the one-CTA budget, then smaller stages.
+    const size_t budgets[2] = {static_cast<size_t>(kGemvSmemTwoCta), static_cast<size_t>(kGemvSmemBudget)};
+    for (size_t budget : budgets) {
+        for (int r = rs; r >= 4; r -= 4) {
+            int st = want < kGemvMaxStages ? want : kGemvMaxStages;
+            if (r != rs) st = (per + r - 1) / r < kGemvMaxStages ? (per + r - 1) / r : kGemvMaxStages;
+            for (; st >= 1; --st) {
+                if (static_cast<size_t>(st) * r * rowbytes + act <= budget) {
+                    if (st < 2 && budget == budgets[0]) break;  // two-CTA plans keep a double buffer
+                    plan->rows_per_stage = r;
+                    plan->stage_bytes = r * rowbytes;
+                    plan->stages = st;
+                    plan->rows_per_cta = per;
+                    plan->grid = static_cast<int>((R + per - 1) / per);
+                    plan->smem_bytes = static_cast<size_t>(st) * plan->stage_bytes + act;
+                    return true;
+                }
+            }
+        }
+    }
+    return false;
 }
 
 __device__ __forceinline__ void gemv_compute_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kGemvComputeWarps * 32) : "memory");
 }
 
+// projection of a global row (row_start is short and sorted)
+__device__ __forceinline__ int gemv_proj_of(const GemvParams& p, int r) {
+    int g = 0;
+#pragma unroll
+    for (int i = 1; i < kGemvMaxProj; ++i)
+        if (i < p.nproj && r >= p.row_start[i]) g = i;
+    return g;
+}
+
 template <int MT, bool FUSED>
-__global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams p) {
+__global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_constant__ GemvParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t full_bar[kGemvStages];
-    __shared__ __align__(8) uint64_t empty_bar[kGemvStages];
+    __shared__ __align__(8) uint64_t full_bar[kGemvMaxStages];
+    __shared__ __align__(8) uint64_t empty_bar[kGemvMaxStages];
     __shared__ __align__(8) uint64_t act_bar;
     __shared__ int qsum_s[MT];
-    __shared__ float cm_s[MT];
+    __shared__ float deq_s[MT];
+    __shared__ float beta_s[kGemvMaxProj];
     __shared__ double red_d[kGemvComputeWarps];
     __shared__ float red_f[kGemvComputeWarps];
     __shared__ int red_i[kGemvComputeWarps];
@@ -106,16 +133,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     const int K = p.K;
     const int rowbytes = K >> 2;
     const int S = p.stages;
+    const int R = p.row_start[p.nproj];
     const int row0 = blockIdx.x * p.rows_per_cta;
-    const int nrows = min(p.N - row0, p.rows_per_cta);
+    const int nrows = min(R - row0, p.rows_per_cta);
     if (nrows <= 0) return;  // uniform for the whole CTA, before any barrier
     const int nst = (nrows + p.rows_per_stage - 1) / p.rows_per_stage;
 
+    // shared memory: [ring: S stages][gamma fp32 K][x bf16 M*K][q int8 M*K]
     uint8_t* ring = smem;
-    uint8_t* act = smem + static_cast<size_t>(S) * p.stage_bytes;
-    const uint16_t* x_s = reinterpret_cast<const uint16_t*>(act);                 // fused: M x K bf16
-    int8_t* q_s = reinterpret_cast<int8_t*>(act + (FUSED ? 2 * static_cast<size_t>(p.M) * K : 0));
-    const uint32_t act_bytes = static_cast<uint32_t>((FUSED ? 2 : 1) * static_cast<size_t>(p.M) * K);
+    float* gamma_s = reinterpret_cast<float*>(smem + static_cast<size_t>(S) * p.stage_bytes);
+    uint16_t* x_s = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(gamma_s) + 4 * static_cast<size_t>(K));
+    int8_t* q_s = reinterpret_cast<int8_t*>(reinterpret_cast<uint8_t*>(x_s) + 2 * static_cast<size_t>(p.M) * K);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -126,24 +154,44 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         abort_flag = 0;
         mbar_fence_init();
     }
+    if (FUSED && threadIdx.x < p.nproj) beta_s[threadIdx.x] = __ldg(p.scale[threadIdx.x]);
     __syncthreads();
 
     if (warp == kGemvComputeWarps) {
-        // ---------------- producer: activations, then packed weight rows -> ring
+        // ---------------- producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(&act_bar, act_bytes);
-            if constexpr (FUSED) bulk_g2s(act, p.x, act_bytes, &act_bar);
-            else bulk_g2s(q_s, p.q_in, act_bytes, &act_bar);
-            const uint8_t* src = reinterpret_cast<const uint8_t*>(p.packed) + static_cast<size_t>(row0) * rowbytes;
-            int issued = 0;
-            for (int s = 0; s < nst; ++s) {
+            auto issue_stage = [&](int s) {
                 const int slot = s % S;
-                if (s >= S && !mbar_wait(&empty_bar[slot], ((s / S) - 1) & 1, &abort_flag)) break;
-                const int r = min(p.rows_per_stage, nrows - s * p.rows_per_stage);
-                const uint32_t bytes = static_cast<uint32_t>(r) * rowbytes;
-                mbar_arrive_expect_tx(&full_bar[slot], bytes);
-                bulk_g2s(ring + static_cast<size_t>(slot) * p.stage_bytes,
-                         src + static_cast<size_t>(s) * p.rows_per_stage * rowbytes, bytes, &full_bar[slot]);
+                const int r0 = row0 + s * p.rows_per_stage;
+                const int r1 = r0 + min(p.rows_per_stage, nrows - s * p.rows_per_stage);
+                mbar_arrive_expect_tx(&full_bar[slot], static_cast<uint32_t>(r1 - r0) * rowbytes);
+                uint8_t* dst = ring + static_cast<size_t>(slot) * p.stage_bytes;
+                for (int r = r0; r < r1;) {  // split at projection boundaries
+                    const int g = gemv_proj_of(p, r);
+                    const int e = min(r1, p.row_start[g + 1]);
+                    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.packed[g]) +
+                                         static_cast<size_t>(r - p.row_start[g]) * rowbytes;
+                    bulk_g2s(dst + static_cast<size_t>(r - r0) * rowbytes, src,
+                             static_cast<uint32_t>(e - r) * rowbytes, &full_bar[slot]);
+                    r = e;
+                }
+            };
+            // weights and gamma are parameters: fetched before the dependency wait
+            const int first = min(nst, S);
+            for (int s = 0; s < first; ++s) issue_stage(s);
+            const uint32_t x_bytes = static_cast<uint32_t>((FUSED ? 2 : 1) * static_cast<size_t>(p.M) * K);
+            const uint32_t g_bytes = FUSED ? 4u * static_cast<uint32_t>(K) : 0u;
+            mbar_arrive_expect_tx(&act_bar, x_bytes + g_bytes);
+            if constexpr (FUSED) bulk_g2s(gamma_s, p.gamma, g_bytes, &act_bar);
+            // activations may come from the previous kernel on the stream
+            pdl_wait();
+            if constexpr (FUSED) bulk_g2s(x_s, p.x, x_bytes, &act_bar);
+            else bulk_g2s(q_s, p.q_in, x_bytes, &act_bar);
+            pdl_launch_dependents();
+            int issued = first;
+            for (int s = first; s < nst; ++s) {
+                if (!mbar_wait(&empty_bar[s % S], ((s / S) - 1) & 1, &abort_flag)) break;
+                issue_stage(s);
                 ++issued;
             }
             // Let every copy this CTA started land before the CTA can exit.
@@ -168,7 +216,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     if constexpr (FUSED) {
         const int C8 = K >> 3;
         const uint4* xr = reinterpret_cast<const uint4*>(x_s + static_cast<size_t>(m) * K);
-        const float4* g4 = reinterpret_cast<const float4*>(p.gamma);
+        const float4* g4 = reinterpret_cast<const float4*>(gamma_s);
         double s2 = 0.0;
         if (active && act_ok) {
             for (int c = tg; c < C8; c += 32 * WPT) {
@@ -195,7 +243,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
             for (int c = tg; c < C8; c += 32 * WPT) {
                 const uint4 v = xr[c];
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
+                const float4 ga = g4[2 * c], gb = g4[2 * c + 1];
                 const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -220,7 +268,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
             for (int c = tg; c < C8; c += 32 * WPT) {
                 const uint4 v = xr[c];
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
+                const float4 ga = g4[2 * c], gb = g4[2 * c + 1];
                 const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
                 uint32_t out[2] = {0u, 0u};
 #pragma unroll
@@ -242,7 +290,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
 #pragma unroll
             for (int i = 0; i < WPT; ++i) t += red_i[w0 + i];
             qsum_s[m] = t;
-            cm_s[m] = __fmul_rn(__fdiv_rn(a, 127.0f), __ldg(p.scale));
+            deq_s[m] = __fdiv_rn(a, 127.0f);
         }
     } else {
         int qs = 0;
@@ -310,7 +358,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
                     }
                 }
             }
-            const int n = row0 + s * p.rows_per_stage + rl;
+            const int r = row0 + s * p.rows_per_stage + rl;
+            const int g = gemv_proj_of(p, valid ? r : row0);
+            const int n = r - p.row_start[g];
+            const int Ng = p.row_start[g + 1] - p.row_start[g];
 #pragma unroll
             for (int mm = 0; mm < MT; ++mm) {
                 int t = acc[mm][0] + (acc[mm][1] >> 2) + (acc[mm][2] >> 4) + (acc[mm][3] >> 6);
@@ -320,10 +371,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
                 if (valid && l8 == 0 && mm < p.M) {
                     const int v = t - qsum_s[mm];
                     if constexpr (FUSED) {
-                        const __nv_bfloat16 yb = __float2bfloat16_rn(__fmul_rn(static_cast<float>(v), cm_s[mm]));
-                        p.y[static_cast<size_t>(mm) * p.N + n] = __bfloat16_as_ushort(yb);
+                        const float cm = __fmul_rn(deq_s[mm], beta_s[g]);
+                        const __nv_bfloat16 yb = __float2bfloat16_rn(__fmul_rn(static_cast<float>(v), cm));
+                        p.y[g][static_cast<size_t>(mm) * Ng + n] = __bfloat16_as_ushort(yb);
                     } else {
-                        p.acc[static_cast<size_t>(mm) * p.N + n] = v;
+                        p.acc[static_cast<size_t>(mm) * Ng + n] = v;
                     }
                 }
             }

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "copy.cuh"
@@ -106,9 +107,31 @@ mmf_status check_shape(int64_t M, int64_t K, int64_t N) {
     return MMF_OK;
 }
 
-bool takes_gemv(int64_t M, int64_t K, int64_t N) {
+bool takes_gemv(int64_t M, int64_t K) {
     GemvPlan plan;
-    return gemv_plan(static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), 148, &plan);
+    return gemv_plan(static_cast<int>(M), static_cast<int>(K), 1, 148, &plan);
+}
+
+// Launches a kernel, as a programmatic dependent of the previous kernel on the
+// stream when `pdl` is set.
+template <typename... KArgs, typename... Args>
+mmf_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                  Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MMF_ERR_CUDA;
+    }
+    return MMF_OK;
 }
 
 int token_tile(int64_t M) {
@@ -164,35 +187,33 @@ mmf_status make_maps(const int8_t* q, const uint32_t* packed, int64_t M, int64_t
 
 template <int BT>
 mmf_status launch_tc_bt(bool fused, const CUtensorMap& mq, const CUtensorMap& mw, const TcParams& p,
-                        cudaStream_t s) {
+                        cudaStream_t s, bool pdl) {
     const dim3 grid(static_cast<unsigned>((p.N + kTcRows - 1) / kTcRows), static_cast<unsigned>((p.M + BT - 1) / BT));
-    if (fused)
-        gemm_tc_kernel<BT, true><<<grid, kTcThreads, TcLayout<BT>::smem_bytes, s>>>(mq, mw, p);
-    else
-        gemm_tc_kernel<BT, false><<<grid, kTcThreads, TcLayout<BT>::smem_bytes, s>>>(mq, mw, p);
-    return launch_status();
+    if (fused) return launch(gemm_tc_kernel<BT, true>, grid, dim3(kTcThreads), TcLayout<BT>::smem_bytes, s, pdl, mq, mw, p);
+    return launch(gemm_tc_kernel<BT, false>, grid, dim3(kTcThreads), TcLayout<BT>::smem_bytes, s, pdl, mq, mw, p);
 }
 
-mmf_status launch_tc(bool fused, const int8_t* q, const uint32_t* packed, const TcParams& p, cudaStream_t s) {
+mmf_status launch_tc(bool fused, const int8_t* q, const uint32_t* packed, const TcParams& p, cudaStream_t s,
+                     bool pdl) {
     const int BT = token_tile(p.M);
     CUtensorMap mq, mw;
     mmf_status st = make_maps(q, packed, p.M, p.K, p.N, BT, &mq, &mw);
     if (st != MMF_OK) return st;
     switch (BT) {
-        case 16: return launch_tc_bt<16>(fused, mq, mw, p, s);
-        case 32: return launch_tc_bt<32>(fused, mq, mw, p, s);
-        case 64: return launch_tc_bt<64>(fused, mq, mw, p, s);
-        case 128: return launch_tc_bt<128>(fused, mq, mw, p, s);
-        default: return launch_tc_bt<256>(fused, mq, mw, p, s);
+        case 16: return launch_tc_bt<16>(fused, mq, mw, p, s, pdl);
+        case 32: return launch_tc_bt<32>(fused, mq, mw, p, s, pdl);
+        case 64: return launch_tc_bt<64>(fused, mq, mw, p, s, pdl);
+        case 128: return launch_tc_bt<128>(fused, mq, mw, p, s, pdl);
+        default: return launch_tc_bt<256>(fused, mq, mw, p, s, pdl);
     }
 }
 
 template <bool FUSED>
-mmf_status launch_gemv(const GemvParams& p, const GemvPlan& plan, cudaStream_t s) {
-    const dim3 grid(static_cast<unsigned>(plan.grid));
+mmf_status launch_gemv(const GemvParams& p, const GemvPlan& plan, cudaStream_t s, bool pdl) {
+    const dim3 grid(static_cast<unsigned>(plan.grid)), block(kGemvThreads);
     switch (p.M) {
 #define MMF_GEMV_CASE(MT) \
-    case MT: gemv_kernel<MT, FUSED><<<grid, kGemvThreads, plan.smem_bytes, s>>>(p); break;
+    case MT: return launch(gemv_kernel<MT, FUSED>, grid, block, plan.smem_bytes, s, pdl, p);
         MMF_GEMV_CASE(1)
         MMF_GEMV_CASE(2)
         MMF_GEMV_CASE(3)
@@ -204,15 +225,66 @@ mmf_status launch_gemv(const GemvParams& p, const GemvPlan& plan, cudaStream_t s
 #undef MMF_GEMV_CASE
         default: return MMF_ERR_UNSUPPORTED_SHAPE;
     }
-    return launch_status();
 }
 
 mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K, int8_t* q,
-                        float* absmax, int* qsum, cudaStream_t s) {
+                        float* absmax, int* qsum, cudaStream_t s, bool pdl) {
     const size_t smem = static_cast<size_t>(K) * 2;
-    rmsnorm_quant_kernel<<<static_cast<unsigned>(M), kQuantThreads, smem, s>>>(x, gamma, eps, static_cast<int>(K), q,
-                                                                                absmax, qsum);
-    return launch_status();
+    return launch(rmsnorm_quant_kernel, dim3(static_cast<unsigned>(M)), dim3(kQuantThreads), smem, s, pdl, x, gamma,
+                  eps, static_cast<int>(K), q, absmax, qsum);
+}
+
+// The fused forward of `count` projections that share x.  Arguments checked.
+mmf_status fwd_impl(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K,
+                    const mmf_projection* proj, int count, void* workspace, unsigned flags, cudaStream_t s,
+                    DeviceState* dev) {
+    const bool pdl = (flags & MMF_FWD_PDL) != 0;
+    int64_t R = 0;
+    for (int i = 0; i < count; ++i) R += proj[i].N;
+    if (R == 0) return MMF_OK;
+    GemvPlan plan;
+    if (gemv_plan(static_cast<int>(M), static_cast<int>(K), R, dev->num_sms, &plan)) {
+        GemvParams p{};
+        p.x = x;
+        p.gamma = gamma;
+        p.eps = eps;
+        p.M = static_cast<int>(M);
+        p.K = static_cast<int>(K);
+        int g = 0;
+        p.row_start[0] = 0;
+        for (int i = 0; i < count; ++i) {
+            if (proj[i].N == 0) continue;
+            p.packed[g] = proj[i].packed;
+            p.scale[g] = proj[i].scale;
+            p.y[g] = proj[i].y;
+            p.row_start[g + 1] = p.row_start[g] + static_cast<int>(proj[i].N);
+            ++g;
+        }
+        p.nproj = g;
+        p.rows_per_stage = plan.rows_per_stage;
+        p.rows_per_cta = plan.rows_per_cta;
+        p.stage_bytes = plan.stage_bytes;
+        p.stages = plan.stages;
+        return launch_gemv<true>(p, plan, s, pdl);
+    }
+    Workspace w = carve(workspace, M, K);
+    mmf_status st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s, pdl);
+    if (st != MMF_OK) return st;
+    for (int i = 0; i < count; ++i) {
+        if (proj[i].N == 0) continue;
+        TcParams p{};
+        p.qsum = w.qsum;
+        p.absmax = w.absmax;
+        p.scale = proj[i].scale;
+        p.y = proj[i].y;
+        p.M = static_cast<int>(M);
+        p.K = static_cast<int>(K);
+        p.N = static_cast<int>(proj[i].N);
+        // only the quantiser may overlap the kernel before it: the contraction
+        // reads the codes the quantiser writes, and waits for it either way
+        if ((st = launch_tc(true, w.q, proj[i].packed, p, s, pdl)) != MMF_OK) return st;
+    }
+    return MMF_OK;
 }
 
 }  // namespace
@@ -242,7 +314,7 @@ size_t mmf_packed_bytes(int64_t N, int64_t K) {
 
 size_t mmf_workspace_bytes(int64_t M, int64_t K, int64_t N) {
     if (check_shape(M, K, N) != MMF_OK || M == 0 || N == 0) return 0;
-    if (takes_gemv(M, K, N)) return 0;
+    if (takes_gemv(M, K)) return 0;
     return workspace_size_tc(M, K);
 }
 
@@ -283,7 +355,7 @@ int mmf_quantize_act(const uint16_t* x, const float* gamma, float eps, int64_t M
     if (!aligned16(x) || !aligned16(gamma) || !aligned16(q) || !aligned16(absmax)) return MMF_ERR_MISALIGNED;
     DeviceState* dev;
     if ((st = device_state(&dev)) != MMF_OK) return st;
-    return launch_quant(x, gamma, eps, M, K, q, absmax, nullptr, static_cast<cudaStream_t>(stream));
+    return launch_quant(x, gamma, eps, M, K, q, absmax, nullptr, static_cast<cudaStream_t>(stream), false);
 }
 
 int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t K, int64_t N, int32_t* acc,
@@ -300,30 +372,33 @@ int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t 
     if ((st = device_state(&dev)) != MMF_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     GemvPlan plan;
-    if (gemv_plan(static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), dev->num_sms, &plan)) {
+    if (gemv_plan(static_cast<int>(M), static_cast<int>(K), N, dev->num_sms, &plan)) {
         GemvParams p{};
         p.q_in = q;
-        p.packed = packed;
+        p.packed[0] = packed;
         p.acc = acc;
+        p.row_start[0] = 0;
+        p.row_start[1] = static_cast<int>(N);
+        p.nproj = 1;
         p.M = static_cast<int>(M);
         p.K = static_cast<int>(K);
-        p.N = static_cast<int>(N);
         p.rows_per_stage = plan.rows_per_stage;
         p.rows_per_cta = plan.rows_per_cta;
         p.stage_bytes = plan.stage_bytes;
         p.stages = plan.stages;
-        return launch_gemv<false>(p, plan, s);
+        return launch_gemv<false>(p, plan, s, false);
     }
     Workspace w = carve(workspace, M, K);
-    qsum_kernel<<<static_cast<unsigned>(M), kQuantThreads, 0, s>>>(q, static_cast<int>(K), w.qsum);
-    if ((st = launch_status()) != MMF_OK) return st;
+    st = launch(qsum_kernel, dim3(static_cast<unsigned>(M)), dim3(kQuantThreads), 0, s, false, q, static_cast<int>(K),
+                w.qsum);
+    if (st != MMF_OK) return st;
     TcParams p{};
     p.qsum = w.qsum;
     p.acc = acc;
     p.M = static_cast<int>(M);
     p.K = static_cast<int>(K);
     p.N = static_cast<int>(N);
-    return launch_tc(false, q, packed, p, s);
+    return launch_tc(false, q, packed, p, s, false);
 }
 
 int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps, const uint32_t* packed, const float* scale,
@@ -341,36 +416,42 @@ int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps, const ui
     if (workspace && !aligned16(workspace)) return MMF_ERR_MISALIGNED;
     DeviceState* dev;
     if ((st = device_state(&dev)) != MMF_OK) return st;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    GemvPlan plan;
-    if (gemv_plan(static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), dev->num_sms, &plan)) {
-        GemvParams p{};
-        p.x = x;
-        p.gamma = gamma;
-        p.eps = eps;
-        p.packed = packed;
-        p.scale = scale;
-        p.y = y;
-        p.M = static_cast<int>(M);
-        p.K = static_cast<int>(K);
-        p.N = static_cast<int>(N);
-        p.rows_per_stage = plan.rows_per_stage;
-        p.rows_per_cta = plan.rows_per_cta;
-        p.stage_bytes = plan.stage_bytes;
-        p.stages = plan.stages;
-        return launch_gemv<true>(p, plan, s);
+    mmf_projection pr;
+    pr.packed = packed;
+    pr.scale = scale;
+    pr.y = y;
+    pr.N = N;
+    return fwd_impl(x, gamma, eps, M, K, &pr, 1, workspace, 0u, static_cast<cudaStream_t>(stream), dev);
+}
+
+int mmf_bitlinear_fwd_group(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K,
+                            const mmf_projection* proj, int count, void* workspace, size_t workspace_bytes,
+                            unsigned flags, void* stream) {
+    if (!(eps >= 0.0f) || eps > 1e30f) return MMF_ERR_INVALID_ARG;
+    if (!proj || count < 1 || count > MMF_MAX_GROUP) return MMF_ERR_INVALID_ARG;
+    if ((flags & ~static_cast<unsigned>(MMF_FWD_PDL)) != 0) return MMF_ERR_INVALID_ARG;
+    int64_t R = 0;
+    for (int i = 0; i < count; ++i) {
+        if (proj[i].N < 0) return MMF_ERR_INVALID_ARG;
+        R += proj[i].N;
     }
-    Workspace w = carve(workspace, M, K);
-    if ((st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s)) != MMF_OK) return st;
-    TcParams p{};
-    p.qsum = w.qsum;
-    p.absmax = w.absmax;
-    p.scale = scale;
-    p.y = y;
-    p.M = static_cast<int>(M);
-    p.K = static_cast<int>(K);
-    p.N = static_cast<int>(N);
-    return launch_tc(true, w.q, packed, p, s);
+    mmf_status st = check_shape(M, K, R);
+    if (st != MMF_OK) return st;
+    if (M == 0 || R == 0) return MMF_OK;
+    if (!x || !gamma) return MMF_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gamma)) return MMF_ERR_MISALIGNED;
+    for (int i = 0; i < count; ++i) {
+        if (proj[i].N == 0) continue;
+        if (!proj[i].packed || !proj[i].scale || !proj[i].y) return MMF_ERR_INVALID_ARG;
+        if (!aligned16(proj[i].packed) || !aligned16(proj[i].scale) || !aligned16(proj[i].y))
+            return MMF_ERR_MISALIGNED;
+    }
+    const size_t need = mmf_workspace_bytes(M, K, R);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return MMF_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return MMF_ERR_MISALIGNED;
+    DeviceState* dev;
+    if ((st = device_state(&dev)) != MMF_OK) return st;
+    return fwd_impl(x, gamma, eps, M, K, proj, count, workspace, flags, static_cast<cudaStream_t>(stream), dev);
 }
 
 int mmf_hbm_copy(const void* src, void* dst, size_t bytes, void* stream) {

@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(kQuantThreads) rmsnorm_quant_kernel(const uint
     __shared__ float red_f[kQuantThreads / 32 + 1];
     __shared__ int red_i[kQuantThreads / 32 + 1];
 
+    pdl_wait();  // x may come from the previous kernel (no-op unless launched as a dependent)
+    pdl_launch_dependents();
     const int64_t m = blockIdx.x;
     const int C = K >> 3;
     const uint4* xr = reinterpret_cast<const uint4*>(x + m * static_cast<int64_t>(K));

@@ -40,10 +40,20 @@ SIGNATURES = {
     "mmf_quantize_act": (_INT, [_P, _P, _F, _I64, _I64, _P, _P, _P]),
     "mmf_ternary_acc": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "mmf_bitlinear_fwd": (_INT, [_P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "mmf_bitlinear_fwd_group": (_INT, [_P, _P, _F, _I64, _I64, _P, _INT, _P, _SZ, C.c_uint, _P]),
     "mmf_hbm_copy": (_INT, [_P, _P, _SZ, _P]),
     "mmf_selftest_timeout": (_INT, [C.c_uint64, _P, _P]),
     "mmf_check_async": (_INT, [_P]),
 }
+
+
+FWD_PDL = 1
+MAX_GROUP = 8
+
+
+class Projection(C.Structure):
+    """mirror of mmf_projection"""
+    _fields_ = [("packed", _P), ("scale", _P), ("y", _P), ("N", _I64)]
 
 
 class MMFError(RuntimeError):
@@ -167,6 +177,29 @@ def bitlinear_fwd(x: torch.Tensor, gamma: torch.Tensor, packed: torch.Tensor, sc
                                   y.data_ptr(), ws.data_ptr() if ws is not None else None, ws_n, _stream(stream)),
           "mmf_bitlinear_fwd")
     return y
+
+
+def projection_array(items):
+    """[(packed, scale, y, N), ...] -> ctypes array of mmf_projection (keep it alive while used)."""
+    arr = (Projection * len(items))()
+    for i, (packed, scale, y, N) in enumerate(items):
+        arr[i] = Projection(packed.data_ptr(), scale.data_ptr(), y.data_ptr() if y is not None else None, N)
+    return arr
+
+
+def bitlinear_fwd_group(x: torch.Tensor, gamma: torch.Tensor, weights, eps: float = 1e-6, workspace=None,
+                        outs=None, flags: int = 0, stream=None):
+    """bf16 x[M, K] and [(packed, scale, N), ...] sharing x -> [bf16 y_i[M, N_i], ...]."""
+    _dev(x, torch.bfloat16, "x")
+    M, K = x.shape
+    ys = outs if outs is not None else [torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+                                        for (_, _, N) in weights]
+    arr = projection_array([(pk, sc, y, N) for (pk, sc, N), y in zip(weights, ys)])
+    ws, ws_n = _workspace(M, K, sum(N for _, _, N in weights), x.device, workspace)
+    check(lib().mmf_bitlinear_fwd_group(x.data_ptr(), gamma.data_ptr(), eps, M, K, arr, len(weights),
+                                        ws.data_ptr() if ws is not None else None, ws_n, flags, _stream(stream)),
+          "mmf_bitlinear_fwd_group")
+    return ys
 
 
 def hbm_copy(src: torch.Tensor, dst: torch.Tensor, stream=None):

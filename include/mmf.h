@@ -141,6 +141,44 @@ int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps,
                       int64_t K, int64_t N, uint16_t* y, void* workspace,
                       size_t workspace_bytes, void* stream);
 
+/* Flags of mmf_bitlinear_fwd_group. */
+#define MMF_FWD_PDL 1u   /* launch as a programmatic dependent of the kernel before it on the stream (see below) */
+#define MMF_MAX_GROUP 8  /* projections per mmf_bitlinear_fwd_group call */
+
+/* One projection of a group: its packed weights and scale (as from
+ * mmf_pack_ternary for an N x K matrix) and its output y, bf16 [M][N]. */
+typedef struct mmf_projection {
+    const uint32_t* packed;
+    const float* scale;
+    uint16_t* y;
+    int64_t N;
+} mmf_projection;
+
+/*
+ * mmf_bitlinear_fwd_group -- the fused forward of `count` (1..MMF_MAX_GROUP)
+ * projections that read the same x: the token mixer's gate projections and
+ * the channel mixer's gate/up pair each share one normalised, quantised input
+ * (jiqizhixin.com, section "MatMul-free 语言模型架构"; datacamp.com, section
+ * "Các thành phần lõi: MLGRU và GLU").  x is normalised and quantised once;
+ * each projection i then gets y_i exactly as mmf_bitlinear_fwd would compute
+ * it (same bits).  On the small-M path all projections run in one launch.
+ *
+ * proj: HOST array of `count` descriptors (read during the call only); an
+ * entry with N == 0 is skipped.  workspace: at least
+ * mmf_workspace_bytes(M, K, sum of N) bytes.
+ *
+ * flags: 0 or MMF_FWD_PDL.  With MMF_FWD_PDL the kernels are launched as
+ * programmatic dependents of the kernel before them on the stream: packed
+ * weights, scales and gamma are fetched BEFORE that kernel has finished (x is
+ * read, and y written, only after it), so the caller guarantees that the
+ * immediately preceding kernel on the stream does not write packed, scale or
+ * gamma.  Without the flag the launches are ordinary stream-ordered launches.
+ */
+int mmf_bitlinear_fwd_group(const uint16_t* x, const float* gamma, float eps,
+                            int64_t M, int64_t K, const mmf_projection* proj,
+                            int count, void* workspace, size_t workspace_bytes,
+                            unsigned flags, void* stream);
+
 /*
  * mmf_hbm_copy -- streaming device-to-device copy of `bytes` bytes (a multiple
  * of 16) with 128-bit loads and stores.  Measurement kernel: it gives the HBM

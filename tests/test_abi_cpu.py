@@ -113,3 +113,23 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(mmf, "LIB_PATH", "/nonexistent/libmmf.so")
     with pytest.raises(RuntimeError, match="missing"):
         mmf.lib()
+
+
+def test_group_argument_errors(L):
+    from bitlinear_rmsnorm_quant_b200 import mmf
+    arr = (mmf.Projection * 1)()
+    arr[0] = mmf.Projection(A, A, A, 16)
+    f = L.mmf_bitlinear_fwd_group
+    assert f(A, A, 1e-6, 1, 128, None, 1, None, 0, 0, None) == 1          # no descriptors
+    assert f(A, A, 1e-6, 1, 128, arr, 0, None, 0, 0, None) == 1           # count 0
+    assert f(A, A, 1e-6, 1, 128, arr, 9, None, 0, 0, None) == 1           # count above the limit
+    assert f(A, A, 1e-6, 1, 128, arr, 1, None, 0, 4, None) == 1           # unknown flag
+    assert f(A, A, 1e-6, 1, 100, arr, 1, None, 0, 0, None) == 2           # bad K
+    arr[0] = mmf.Projection(A, A, None, 16)
+    assert f(A, A, 1e-6, 1, 128, arr, 1, None, 0, 0, None) == 1           # null y
+    arr[0] = mmf.Projection(A, MIS, A, 16)
+    assert f(A, A, 1e-6, 1, 128, arr, 1, None, 0, 1, None) == 3           # misaligned scale
+    arr[0] = mmf.Projection(None, None, None, 0)
+    assert f(None, None, 1e-6, 1, 128, arr, 1, None, 0, 0, None) == 0     # empty group
+    arr[0] = mmf.Projection(A, A, A, 16)
+    assert f(A, A, 1e-6, 4096, 2048, arr, 1, None, 0, 0, None) == 4       # large M needs workspace

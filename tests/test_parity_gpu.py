@@ -234,6 +234,51 @@ def test_fwd_deterministic():
         assert torch.equal(y1, y2)
 
 
+# -- grouped projections sharing x -------------------------------------------------------------
+
+@pytest.mark.parametrize("M,K,Ns", [(1, 2560, (2560, 2560, 2560, 2560)), (1, 2560, (6912, 6912)),
+                                    (3, 1024, (100, 0, 333, 64)), (8, 512, (128,) * 8),
+                                    (64, 1024, (300, 129)), (300, 384, (256, 200, 17))])
+@pytest.mark.parametrize("flags", [0, 1])
+def test_group_matches_single_calls(oracle, M, K, Ns, flags):
+    x, g, _ = make_layer(14, M, K, 1)
+    xd, gd = x.to(DEV), g.to(DEV)
+    weights, Ws = [], []
+    for i, N in enumerate(Ns):
+        W = make_layer(14, 1, K, max(N, 1), index=i + 1)[2][:N]
+        Ws.append(W)
+        packed, scale = _pack(W.contiguous()) if N > 0 else (torch.zeros(1, K // 16, dtype=torch.int32, device=DEV),
+                                                             torch.ones(1, device=DEV))
+        weights.append((packed, scale, N))
+    ys = mmf.bitlinear_fwd_group(xd, gd, weights, EPS, flags=flags)
+    singles = [mmf.bitlinear_fwd(xd, gd, pk, sc, N, EPS) if N > 0 else None for (pk, sc, N) in weights]
+    torch.cuda.synchronize()
+    for (pk, sc, N), y, y1, W in zip(weights, ys, singles, Ws):
+        assert y.shape == (M, N)
+        if N == 0:
+            continue
+        assert torch.equal(y, y1)
+        y_ref, _ = oracle.bitlinear(bits_np(x), g.numpy(), EPS, W.contiguous().numpy(), EPS_W)
+        assert y_rel_error(bits_np(y), y_ref) <= Y_REL_TOL
+
+
+def test_group_pdl_chain_matches_plain():
+    """A chain of PDL launches in one stream gives the same bits as plain launches."""
+    K = 2048
+    x, g, _ = make_layer(15, 1, K, 1)
+    xd, gd = x.to(DEV), g.to(DEV)
+    weights = []
+    for i in range(6):
+        W = make_layer(15, 1, K, 1024, index=i + 1)[2]
+        pk, sc = _pack(W)
+        weights.append((pk, sc, 1024))
+    plain = [mmf.bitlinear_fwd_group(xd, gd, [w], EPS)[0] for w in weights]
+    chained = [mmf.bitlinear_fwd_group(xd, gd, [w], EPS, flags=mmf.FWD_PDL)[0] for w in weights]
+    torch.cuda.synchronize()
+    for a, b in zip(plain, chained):
+        assert torch.equal(a, b)
+
+
 # -- error paths on the device -----------------------------------------------------------------
 
 def test_argument_errors_on_device():
