@@ -15,29 +15,36 @@
 // power-of-four lanes are shifted back and summed once per row, and the
 // per-token sum_k q_k is subtracted once.  All integer, exact.
 //
-// CTA: 8 compute warps + 1 producer warp.  The group's weight rows form one
+// CTA: 16 compute warps (8 when M > 4) + 1 producer warp.  The group's weight rows form one
 // concatenated row space; each CTA owns a contiguous range of it.  The
 // producer bulk-copies (TMA) the CTA's weight rows into a ring of small
 // shared-memory stages and gamma into shared memory, then waits for the
 // previous kernel on the stream (programmatic dependent launch; a no-op when
 // the launch is not programmatic), then copies the M rows of x.  So under PDL
 // the weight stream overlaps the previous kernel and only x waits for it.
-// Compute warps take groups of 4 rows; 8 lanes cover one row, lane l reading
-// 16-byte chunks l, l+8, ... (64 weights each); a row's 8 partials meet in a
-// 3-step warp-shuffle tree.
+// Compute warps take blocks of 8 rows, round-robin over the whole slab (so
+// every warp works whatever the stage size); lane (r, l) of a warp covers rows
+// r and r+4 of the block, reading their 16-byte chunks l, l+8, ... (64 weights
+// each) against one shared load of the activation codes; a row's 8 partials
+// meet in a 3-step warp-shuffle tree.
 #pragma once
 #include "common.cuh"
 
 namespace mmf {
 
-constexpr int kGemvComputeWarps = 8;
-constexpr int kGemvThreads = (kGemvComputeWarps + 1) * 32;
+constexpr int kGemvMaxComputeWarps = 16;
+
+// compute warps per CTA: 16 while the accumulators are few enough for the
+// register file (M <= 4), else 8; plus one producer warp
+__host__ __device__ constexpr int gemv_compute_warps(int M) { return M <= 4 ? 16 : 8; }
+__host__ __device__ constexpr int gemv_threads(int M) { return (gemv_compute_warps(M) + 1) * 32; }
 constexpr int kGemvMaxStages = 8;
 constexpr int kGemvMaxTokens = 8;
 constexpr int kGemvMaxProj = 8;
-constexpr int kGemvStageTarget = 8192;       // bytes of packed weights per stage
+constexpr int kGemvStageTarget = 10240;      // bytes of packed weights per stage
+constexpr int kGemvBlockRows = 8;            // rows per warp work item
 constexpr int kGemvSmemTwoCta = 110 * 1024;  // two CTAs per SM fit under this
-constexpr int kGemvSmemBudget = 200 * 1024;
+constexpr int kGemvSmemBudget = 220 * 1024;   // under the 227 KB per-CTA limit with the static part
 
 struct GemvParams {
     const uint16_t* x;                      // bf16 [M][K]      (fused mode)
@@ -50,7 +57,7 @@ struct GemvParams {
     int row_start[kGemvMaxProj + 1];        // prefix sums of N_g
     float eps;
     int M, K, nproj;
-    int rows_per_stage;                     // multiple of 4
+    int rows_per_stage;                     // multiple of kGemvBlockRows
     int rows_per_cta;
     int stage_bytes;                        // rows_per_stage * K/4
     int stages;                             // 1 .. kGemvMaxStages
@@ -70,19 +77,19 @@ inline bool gemv_plan(int M, int K, int64_t R, int num_sms, GemvPlan* plan) {
     if (M < 1 || M > kGemvMaxTokens || R < 1) return false;
     const int rowbytes = K / 4;
     const size_t act = gemv_act_bytes(M, K);
-    int rs = 4 * (kGemvStageTarget / (4 * rowbytes));
-    if (rs < 4) rs = 4;
+    constexpr int B = kGemvBlockRows;
+    int rs = B * (kGemvStageTarget / (B * rowbytes));
+    if (rs < B) rs = B;
     if (rs > 64) rs = 64;
-    int grid = static_cast<int>((R + 3) / 4);
+    int grid = static_cast<int>((R + B - 1) / B);
     if (grid > num_sms) grid = num_sms;
-    int per = static_cast<int>((R + grid - 1) / grid);
-    per = (per + 3) & ~3;
+    const int per = static_cast<int>((R + grid - 1) / grid);  // blocks may be partial
     const int want = (per + rs - 1) / rs;  // stages that hold the CTA's whole slab
     // Prefer a ring that holds the whole slab within the two-CTA budget, then
     // fewer stages, then the one-CTA budget, then smaller stages.
     const size_t budgets[2] = {static_cast<size_t>(kGemvSmemTwoCta), static_cast<size_t>(kGemvSmemBudget)};
     for (size_t budget : budgets) {
-        for (int r = rs; r >= 4; r -= 4) {
+        for (int r = rs; r >= B; r -= B) {
             int st = want < kGemvMaxStages ? want : kGemvMaxStages;
             if (r != rs) st = (per + r - 1) / r < kGemvMaxStages ? (per + r - 1) / r : kGemvMaxStages;
             for (; st >= 1; --st) {
@@ -102,8 +109,23 @@ inline bool gemv_plan(int M, int K, int64_t R, int num_sms, GemvPlan* plan) {
     return false;
 }
 
+// Fixed-shape pairwise combine of n (a power of two) per-warp partials: the
+// same tree every run, so the fp64 sum is deterministic.
+template <int n, typename T>
+__device__ __forceinline__ T tree_sum(const T* v) {
+    if constexpr (n == 1) return v[0];
+    else return tree_sum<n / 2>(v) + tree_sum<n / 2>(v + n / 2);
+}
+
+template <int n>
+__device__ __forceinline__ float tree_max(const float* v) {
+    if constexpr (n == 1) return v[0];
+    else return fmaxf(tree_max<n / 2>(v), tree_max<n / 2>(v + n / 2));
+}
+
+template <int NW>
 __device__ __forceinline__ void gemv_compute_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kGemvComputeWarps * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
 }
 
 // projection of a global row (row_start is short and sorted)
@@ -115,8 +137,10 @@ __device__ __forceinline__ int gemv_proj_of(const GemvParams& p, int r) {
     return g;
 }
 
+// One CTA per SM: the register file goes to independent accumulator chains.
 template <int MT, bool FUSED>
-__global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_constant__ GemvParams p) {
+__global__ void __launch_bounds__(gemv_threads(MT), 1) gemv_kernel(const __grid_constant__ GemvParams p) {
+    constexpr int NW = gemv_compute_warps(MT);
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t full_bar[kGemvMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kGemvMaxStages];
@@ -124,9 +148,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     __shared__ int qsum_s[MT];
     __shared__ float deq_s[MT];
     __shared__ float beta_s[kGemvMaxProj];
-    __shared__ double red_d[kGemvComputeWarps];
-    __shared__ float red_f[kGemvComputeWarps];
-    __shared__ int red_i[kGemvComputeWarps];
+    __shared__ double red_d[NW];
+    __shared__ float red_f[NW];
+    __shared__ int red_i[NW];
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -139,7 +163,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     if (nrows <= 0) return;  // uniform for the whole CTA, before any barrier
     const int nst = (nrows + p.rows_per_stage - 1) / p.rows_per_stage;
 
-    // shared memory: [ring: S stages][gamma fp32 K][x bf16 M*K][q int8 M*K]
+    // shared memory: [ring: S stages][gamma fp32 K][x bf16 M*K][q int8 M*K].
+    // q is stored t-major: the 16 codes k = 64c + 16t .. +15 sit at 16*(t*C + c)
+    // (C = K/64), so the 8 lanes of a row read 128 contiguous bytes at each t.
     uint8_t* ring = smem;
     float* gamma_s = reinterpret_cast<float*>(smem + static_cast<size_t>(S) * p.stage_bytes);
     uint16_t* x_s = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(gamma_s) + 4 * static_cast<size_t>(K));
@@ -148,16 +174,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], kGemvComputeWarps);
+            mbar_init(&empty_bar[s], NW);
         }
         mbar_init(&act_bar, 1);
         abort_flag = 0;
         mbar_fence_init();
     }
-    if (FUSED && threadIdx.x < p.nproj) beta_s[threadIdx.x] = __ldg(p.scale[threadIdx.x]);
     __syncthreads();
 
-    if (warp == kGemvComputeWarps) {
+    if (warp == NW) {
         // ---------------- producer
         if (lane == 0) {
             auto issue_stage = [&](int s) {
@@ -176,17 +201,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
                     r = e;
                 }
             };
-            // weights and gamma are parameters: fetched before the dependency wait
-            const int first = min(nst, S);
-            for (int s = 0; s < first; ++s) issue_stage(s);
+            // gamma and the weights are parameters: fetched before the dependency
+            // wait (gamma first, the normalisation needs it before any weight)
             const uint32_t x_bytes = static_cast<uint32_t>((FUSED ? 2 : 1) * static_cast<size_t>(p.M) * K);
             const uint32_t g_bytes = FUSED ? 4u * static_cast<uint32_t>(K) : 0u;
             mbar_arrive_expect_tx(&act_bar, x_bytes + g_bytes);
             if constexpr (FUSED) bulk_g2s(gamma_s, p.gamma, g_bytes, &act_bar);
+            const int first = min(nst, S);
+            for (int s = 0; s < first; ++s) issue_stage(s);
             // activations may come from the previous kernel on the stream
             pdl_wait();
-            if constexpr (FUSED) bulk_g2s(x_s, p.x, x_bytes, &act_bar);
-            else bulk_g2s(q_s, p.q_in, x_bytes, &act_bar);
+            bulk_g2s(x_s, FUSED ? static_cast<const void*>(p.x) : static_cast<const void*>(p.q_in), x_bytes, &act_bar);
             pdl_launch_dependents();
             int issued = first;
             for (int s = first; s < nst; ++s) {
@@ -203,15 +228,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     }
 
     // ---------------- compute warps: RMSNorm + int8 quantisation of the M tokens.
-    // Token m is shared by WPT = 8 / MP warps (MP = M rounded up to a power of
+    // Token m is shared by WPT = NW / MP warps (MP = M rounded up to a power of
     // two); every reduction is per-thread sequential, a warp xor-tree, then the
     // group's warps in index order, so the result does not vary run to run.
     constexpr int MP = MT <= 1 ? 1 : (MT <= 2 ? 2 : (MT <= 4 ? 4 : 8));
-    constexpr int WPT = kGemvComputeWarps / MP;
+    constexpr int WPT = NW / MP;
     const int m = warp / WPT;
     const bool active = m < p.M;
     const int tg = (warp % WPT) * 32 + lane;
     const int w0 = m * WPT;
+    if (FUSED && threadIdx.x < p.nproj) beta_s[threadIdx.x] = __ldg(p.scale[threadIdx.x]);  // read after a compute sync
     const bool act_ok = mbar_wait(&act_bar, 0, &abort_flag);
     if constexpr (FUSED) {
         const int C8 = K >> 3;
@@ -231,10 +257,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
         }
         s2 = warp_sum_f64(s2);
         if (lane == 0) red_d[warp] = s2;
-        gemv_compute_sync();
-        s2 = 0.0;
-#pragma unroll
-        for (int i = 0; i < WPT; ++i) s2 += red_d[(w0 + i) % kGemvComputeWarps];
+        gemv_compute_sync<NW>();
+        s2 = tree_sum<WPT>(red_d + w0);
         const float ms = static_cast<float>(s2 / static_cast<double>(K));
         const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.eps)));
 
@@ -253,18 +277,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
                 }
             }
         }
-        amax = warp_max_f32(amax);
+        amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));  // amax >= 0
         if (lane == 0) red_f[warp] = amax;
-        gemv_compute_sync();
-        amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < WPT; ++i) amax = fmaxf(amax, red_f[(w0 + i) % kGemvComputeWarps]);
+        gemv_compute_sync<NW>();
+        amax = tree_max<WPT>(red_f + w0);
         const float a = fmaxf(amax, 1e-5f);
         const float s = __fdiv_rn(127.0f, a);
 
         int qs = 0;
         if (active && act_ok) {
-            uint2* qrow = reinterpret_cast<uint2*>(q_s + static_cast<size_t>(m) * K);
+            int8_t* qrow = q_s + static_cast<size_t>(m) * K;
+            const int C64 = K >> 6;
             for (int c = tg; c < C8; c += 32 * WPT) {
                 const uint4 v = xr[c];
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -279,92 +302,136 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
                     qs += code;
                     out[i >> 2] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (i & 3));
                 }
-                qrow[c] = make_uint2(out[0], out[1]);
+                // codes k = 8c .. 8c+7 -> unit (c/8, (c%8)/2), half c%2 of the t-major layout
+                *reinterpret_cast<uint2*>(qrow + 16 * (((c & 7) >> 1) * C64 + (c >> 3)) + 8 * (c & 1)) =
+                    make_uint2(out[0], out[1]);
             }
         }
-        qs = warp_sum_i32(qs);
+        qs = __reduce_add_sync(0xffffffffu, qs);
         if (lane == 0) red_i[warp] = qs;
-        gemv_compute_sync();
+        gemv_compute_sync<NW>();
         if (active && tg == 0) {
-            int t = 0;
-#pragma unroll
-            for (int i = 0; i < WPT; ++i) t += red_i[w0 + i];
-            qsum_s[m] = t;
+            qsum_s[m] = tree_sum<WPT>(red_i + w0);
             deq_s[m] = __fdiv_rn(a, 127.0f);
         }
     } else {
         int qs = 0;
         if (active && act_ok) {
-            const uint4* qr = reinterpret_cast<const uint4*>(q_s + static_cast<size_t>(m) * K);
+            // codes arrive in natural order in the x area; 16-byte unit u = 4c + t
+            // moves to position t*C + c of the t-major layout
+            const uint4* qr = reinterpret_cast<const uint4*>(reinterpret_cast<const int8_t*>(x_s) +
+                                                             static_cast<size_t>(m) * K);
+            uint4* qrow = reinterpret_cast<uint4*>(q_s + static_cast<size_t>(m) * K);
+            const int C64 = K >> 6;
             for (int c = tg; c < (K >> 4); c += 32 * WPT) {
                 const uint4 v = qr[c];
+                qrow[(c & 3) * C64 + (c >> 2)] = v;
                 qs = __dp4a(static_cast<int>(v.x), 0x01010101, qs);
                 qs = __dp4a(static_cast<int>(v.y), 0x01010101, qs);
                 qs = __dp4a(static_cast<int>(v.z), 0x01010101, qs);
                 qs = __dp4a(static_cast<int>(v.w), 0x01010101, qs);
             }
         }
-        qs = warp_sum_i32(qs);
+        qs = __reduce_add_sync(0xffffffffu, qs);
         if (lane == 0) red_i[warp] = qs;
-        gemv_compute_sync();
+        gemv_compute_sync<NW>();
         if (active && tg == 0) {
-            int t = 0;
-#pragma unroll
-            for (int i = 0; i < WPT; ++i) t += red_i[w0 + i];
-            qsum_s[m] = t;
+            qsum_s[m] = tree_sum<WPT>(red_i + w0);
         }
     }
-    gemv_compute_sync();
+    gemv_compute_sync<NW>();
     if (!act_ok) return;
 
     // ---------------- contraction over the staged rows
-    const int g_row = lane >> 3;  // row within a group of 4
-    const int l8 = lane & 7;      // lane within the row
-    const int C = K >> 6;         // 16-byte chunks (64 weights) per row
-    for (int s = 0; s < nst; ++s) {
-        const int slot = s % S;
-        const bool ok = mbar_wait(&full_bar[slot], (s / S) & 1, &abort_flag);
-        if (!ok) break;
+    // Blocks of 8 rows go round-robin to the compute warps over the whole slab.
+    const int rsub = lane >> 3;    // lane handles rows rsub and rsub + 4 of a block
+    const int l8 = lane & 7;       // lane within the row
+    const int C = K >> 6;          // 16-byte chunks (64 weights) per row
+    const int bps = p.rows_per_stage / kGemvBlockRows;
+    const int nblocks = (nrows + kGemvBlockRows - 1) / kGemvBlockRows;
+
+    auto do_block = [&](int gb, int s, int slot) {
         const int rs = min(p.rows_per_stage, nrows - s * p.rows_per_stage);
-        const int ngroups = (rs + 3) >> 2;
+        const int b = gb - s * bps;
         const uint8_t* stage = ring + static_cast<size_t>(slot) * p.stage_bytes;
-        for (int grp = warp; grp < ngroups; grp += kGemvComputeWarps) {
-            const int rl = 4 * grp + g_row;
-            const bool valid = rl < rs;
-            int acc[MT][4];
+        const int rl0 = kGemvBlockRows * b + rsub, rl1 = rl0 + 4;
+        const bool v0 = rl0 < rs, v1 = rl1 < rs;
+        int acc0[MT][4], acc1[MT][4];
+        const uint4* w0p = reinterpret_cast<const uint4*>(stage + static_cast<size_t>(v0 ? rl0 : 0) * rowbytes);
+        const uint4* w1p = reinterpret_cast<const uint4*>(stage + static_cast<size_t>(v1 ? rl1 : 0) * rowbytes);
+        if constexpr (MT == 1) {
+            // one token: separate accumulators per (row, t, j), 32 independent
+            // DP4A chains per lane, summed once after the loop
+            int a[2][4][4];
 #pragma unroll
-            for (int mm = 0; mm < MT; ++mm)
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[mm][j] = 0;
-            if (valid) {
-                const uint4* wrow = reinterpret_cast<const uint4*>(stage + static_cast<size_t>(rl) * rowbytes);
+                for (int t = 0; t < 4; ++t)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) a[h][t][j] = 0;
 #pragma unroll 2
-                for (int c = l8; c < C; c += 8) {
-                    const uint4 wv = wrow[c];
-                    const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+            for (int c = l8; c < C; c += 8) {
+                const uint4 wa = w0p[c], wb = w1p[c];
+                const uint32_t da[4] = {wa.x, wa.y, wa.z, wa.w};
+                const uint32_t db[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const uint32_t m0 = wd[t] & 0x03030303u, m1 = wd[t] & 0x0C0C0C0Cu;
-                        const uint32_t m2 = wd[t] & 0x30303030u, m3 = wd[t] & 0xC0C0C0C0u;
-#pragma unroll
-                        for (int mm = 0; mm < MT; ++mm) {
-                            const uint4 qv =
-                                *reinterpret_cast<const uint4*>(q_s + static_cast<size_t>(mm) * K + 64 * c + 16 * t);
-                            acc[mm][0] = dp4a_us(m0, qv.x, acc[mm][0]);
-                            acc[mm][1] = dp4a_us(m1, qv.y, acc[mm][1]);
-                            acc[mm][2] = dp4a_us(m2, qv.z, acc[mm][2]);
-                            acc[mm][3] = dp4a_us(m3, qv.w, acc[mm][3]);
-                        }
-                    }
+                for (int t = 0; t < 4; ++t) {
+                    const uint4 qv = *reinterpret_cast<const uint4*>(q_s + 16 * (t * C + c));
+                    a[0][t][0] = dp4a_us(da[t] & 0x03030303u, qv.x, a[0][t][0]);
+                    a[0][t][1] = dp4a_us(da[t] & 0x0C0C0C0Cu, qv.y, a[0][t][1]);
+                    a[0][t][2] = dp4a_us(da[t] & 0x30303030u, qv.z, a[0][t][2]);
+                    a[0][t][3] = dp4a_us(da[t] & 0xC0C0C0C0u, qv.w, a[0][t][3]);
+                    a[1][t][0] = dp4a_us(db[t] & 0x03030303u, qv.x, a[1][t][0]);
+                    a[1][t][1] = dp4a_us(db[t] & 0x0C0C0C0Cu, qv.y, a[1][t][1]);
+                    a[1][t][2] = dp4a_us(db[t] & 0x30303030u, qv.z, a[1][t][2]);
+                    a[1][t][3] = dp4a_us(db[t] & 0xC0C0C0C0u, qv.w, a[1][t][3]);
                 }
             }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                acc0[0][j] = (a[0][0][j] + a[0][1][j]) + (a[0][2][j] + a[0][3][j]);
+                acc1[0][j] = (a[1][0][j] + a[1][1][j]) + (a[1][2][j] + a[1][3][j]);
+            }
+        } else {
+#pragma unroll
+        for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc0[mm][j] = acc1[mm][j] = 0;
+#pragma unroll 2
+        for (int c = l8; c < C; c += 8) {
+            const uint4 wa = w0p[c], wb = w1p[c];
+            const uint32_t da[4] = {wa.x, wa.y, wa.z, wa.w};
+            const uint32_t db[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const uint32_t a0 = da[t] & 0x03030303u, a1 = da[t] & 0x0C0C0C0Cu;
+                const uint32_t a2 = da[t] & 0x30303030u, a3 = da[t] & 0xC0C0C0C0u;
+                const uint32_t c0 = db[t] & 0x03030303u, c1 = db[t] & 0x0C0C0C0Cu;
+                const uint32_t c2 = db[t] & 0x30303030u, c3 = db[t] & 0xC0C0C0C0u;
+#pragma unroll
+                for (int mm = 0; mm < MT; ++mm) {
+                    const uint4 qv =
+                        *reinterpret_cast<const uint4*>(q_s + static_cast<size_t>(mm) * K + 16 * (t * C + c));
+                    acc0[mm][0] = dp4a_us(a0, qv.x, acc0[mm][0]);
+                    acc0[mm][1] = dp4a_us(a1, qv.y, acc0[mm][1]);
+                    acc0[mm][2] = dp4a_us(a2, qv.z, acc0[mm][2]);
+                    acc0[mm][3] = dp4a_us(a3, qv.w, acc0[mm][3]);
+                    acc1[mm][0] = dp4a_us(c0, qv.x, acc1[mm][0]);
+                    acc1[mm][1] = dp4a_us(c1, qv.y, acc1[mm][1]);
+                    acc1[mm][2] = dp4a_us(c2, qv.z, acc1[mm][2]);
+                    acc1[mm][3] = dp4a_us(c3, qv.w, acc1[mm][3]);
+                }
+            }
+        }
+        }
+        auto finish_row = [&](const int (&ac)[MT][4], int rl, bool valid) {
             const int r = row0 + s * p.rows_per_stage + rl;
             const int g = gemv_proj_of(p, valid ? r : row0);
             const int n = r - p.row_start[g];
             const int Ng = p.row_start[g + 1] - p.row_start[g];
 #pragma unroll
             for (int mm = 0; mm < MT; ++mm) {
-                int t = acc[mm][0] + (acc[mm][1] >> 2) + (acc[mm][2] >> 4) + (acc[mm][3] >> 6);
+                int t = ac[mm][0] + (ac[mm][1] >> 2) + (ac[mm][2] >> 4) + (ac[mm][3] >> 6);
                 t += __shfl_xor_sync(0xffffffffu, t, 1);
                 t += __shfl_xor_sync(0xffffffffu, t, 2);
                 t += __shfl_xor_sync(0xffffffffu, t, 4);
@@ -379,9 +446,33 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
                     }
                 }
             }
+        };
+        finish_row(acc0, rl0, v0);
+        finish_row(acc1, rl1, v1);
+    };
+
+    if (nst <= S) {
+        // The ring holds the whole slab: every slot is filled once (phase 0),
+        // so a warp waits only for the stage of each of its blocks.
+        for (int gb = warp; gb < nblocks; gb += NW) {
+            const int s = gb / bps;
+            if (!mbar_wait(&full_bar[s], 0, &abort_flag)) break;
+            do_block(gb, s, s);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[slot]);
+    } else {
+        // Slots are refilled: every warp walks the stages in order and releases
+        // each one (a parity wait only tells adjacent phases apart, so no warp
+        // may look at a slot more than one phase ahead of its last release).
+        for (int s = 0; s < nst; ++s) {
+            const int slot = s % S;
+            if (!mbar_wait(&full_bar[slot], (s / S) & 1, &abort_flag)) break;
+            const int nb = (min(p.rows_per_stage, nrows - s * p.rows_per_stage) + kGemvBlockRows - 1) / kGemvBlockRows;
+            int first = warp - (s * bps) % NW;  // first block of this stage owned by this warp
+            if (first < 0) first += NW;
+            for (int b = first; b < nb; b += NW) do_block(s * bps + b, s, slot);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[slot]);
+        }
     }
 }
 

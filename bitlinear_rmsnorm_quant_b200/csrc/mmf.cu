@@ -210,10 +210,10 @@ mmf_status launch_tc(bool fused, const int8_t* q, const uint32_t* packed, const 
 
 template <bool FUSED>
 mmf_status launch_gemv(const GemvParams& p, const GemvPlan& plan, cudaStream_t s, bool pdl) {
-    const dim3 grid(static_cast<unsigned>(plan.grid)), block(kGemvThreads);
+    const dim3 grid(static_cast<unsigned>(plan.grid));
     switch (p.M) {
 #define MMF_GEMV_CASE(MT) \
-    case MT: return launch(gemv_kernel<MT, FUSED>, grid, block, plan.smem_bytes, s, pdl, p);
+    case MT: return launch(gemv_kernel<MT, FUSED>, grid, dim3(gemv_threads(MT)), plan.smem_bytes, s, pdl, p);
         MMF_GEMV_CASE(1)
         MMF_GEMV_CASE(2)
         MMF_GEMV_CASE(3)

@@ -110,6 +110,7 @@ def test_quantize_special_rows(oracle):
 ACC_SHAPES = [
     # (M, K, N) decode GEMV path (M <= 8)
     (1, 128, 1), (1, 256, 256), (2, 1024, 1000), (3, 2560, 333), (8, 6912, 2560), (5, 2816, 1024),
+    (1, 6912, 20000), (4, 4096, 9000),   # weight ring refilled many times per CTA
     # tcgen05 path: several 128-row tiles, token tiles, K stages, ragged tails
     (9, 256, 300), (16, 256, 256), (17, 384, 129), (32, 2560, 640), (100, 1024, 257), (256, 512, 384),
     (300, 384, 300), (513, 2048, 200),
@@ -162,7 +163,7 @@ def _layer_parity(oracle, x, g, W, sample_tokens=None):
     return err
 
 
-@pytest.mark.parametrize("M,K,N", [(1, 128, 16), (1, 1024, 2816), (4, 2560, 1000), (8, 6912, 2560),
+@pytest.mark.parametrize("M,K,N", [(1, 128, 16), (1, 1024, 2816), (4, 2560, 1000), (8, 6912, 2560), (1, 6912, 20000),
                                    (9, 256, 256), (16, 256, 256), (33, 2048, 500), (300, 384, 300),
                                    (1000, 1024, 384)])
 def test_bitlinear_parity(oracle, M, K, N):
