@@ -32,6 +32,15 @@ std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 
+// Scratch of mmf_bitlinear_fwd_noalloc: the large-M workspace (int8 codes,
+// absmax, per-token sums) lives here instead of in caller memory.  Every GPU
+// that loads the library holds these bytes until the process exits.
+constexpr size_t kNoAllocScratchBytes = MMF_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+// Device address of g_noalloc_scratch on each device (host code cannot use the
+// symbol's name as an address); filled on the first call on that device.
+void* g_noalloc_scratch_ptr[kMaxDevices];
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -452,6 +461,42 @@ int mmf_bitlinear_fwd_group(const uint16_t* x, const float* gamma, float eps, in
     DeviceState* dev;
     if ((st = device_state(&dev)) != MMF_OK) return st;
     return fwd_impl(x, gamma, eps, M, K, proj, count, workspace, flags, static_cast<cudaStream_t>(stream), dev);
+}
+
+int mmf_bitlinear_fwd_noalloc(const uint16_t* x, const float* gamma, float eps, const uint32_t* packed,
+                              const float* scale, int64_t M, int64_t K, int64_t N, uint16_t* y, void* stream) {
+    if (!(eps >= 0.0f) || eps > 1e30f) return MMF_ERR_INVALID_ARG;
+    mmf_status st = check_shape(M, K, N);
+    if (st != MMF_OK) return st;
+    if (M == 0 || N == 0) return MMF_OK;
+    if (!x || !gamma || !packed || !scale || !y) return MMF_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gamma) || !aligned16(packed) || !aligned16(scale) || !aligned16(y))
+        return MMF_ERR_MISALIGNED;
+    const size_t need = mmf_workspace_bytes(M, K, N);
+    if (need > kNoAllocScratchBytes) return MMF_ERR_WORKSPACE;  // larger than the static scratch
+    DeviceState* dev;
+    if ((st = device_state(&dev)) != MMF_OK) return st;
+    void* ws = nullptr;
+    if (need > 0) {
+        int d = 0;
+        if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return MMF_ERR_NO_DEVICE;
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!g_noalloc_scratch_ptr[d]) {
+            // once per device, with that device current
+            void* ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MMF_ERR_CUDA;
+            g_noalloc_scratch_ptr[d] = ptr;
+        }
+        ws = g_noalloc_scratch_ptr[d];
+    }
+    // Nothing in the scratch has to start at zero: the quantiser writes every
+    // code, absmax and sum the contraction reads, on each call.
+    mmf_projection pr;
+    pr.packed = packed;
+    pr.scale = scale;
+    pr.y = y;
+    pr.N = N;
+    return fwd_impl(x, gamma, eps, M, K, &pr, 1, ws, 0u, static_cast<cudaStream_t>(stream), dev);
 }
 
 int mmf_hbm_copy(const void* src, void* dst, size_t bytes, void* stream) {

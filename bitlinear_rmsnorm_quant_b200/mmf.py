@@ -41,6 +41,7 @@ SIGNATURES = {
     "mmf_ternary_acc": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "mmf_bitlinear_fwd": (_INT, [_P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "mmf_bitlinear_fwd_group": (_INT, [_P, _P, _F, _I64, _I64, _P, _INT, _P, _SZ, C.c_uint, _P]),
+    "mmf_bitlinear_fwd_noalloc": (_INT, [_P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P]),
     "mmf_hbm_copy": (_INT, [_P, _P, _SZ, _P]),
     "mmf_selftest_timeout": (_INT, [C.c_uint64, _P, _P]),
     "mmf_check_async": (_INT, [_P]),
@@ -48,6 +49,7 @@ SIGNATURES = {
 
 
 FWD_PDL = 1
+NOALLOC_SCRATCH_BYTES = 64 << 20   # MMF_NOALLOC_SCRATCH_BYTES
 MAX_GROUP = 8
 
 
@@ -200,6 +202,19 @@ def bitlinear_fwd_group(x: torch.Tensor, gamma: torch.Tensor, weights, eps: floa
                                         ws.data_ptr() if ws is not None else None, ws_n, flags, _stream(stream)),
           "mmf_bitlinear_fwd_group")
     return ys
+
+
+def bitlinear_fwd_noalloc(x: torch.Tensor, gamma: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, N: int,
+                          eps: float = 1e-6, out: torch.Tensor | None = None, stream=None):
+    """As bitlinear_fwd, but the library's static scratch replaces the workspace
+    (for callers that cannot allocate device memory; pass `out` to allocate
+    nothing here either)."""
+    _dev(x, torch.bfloat16, "x")
+    M, K = x.shape
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    check(lib().mmf_bitlinear_fwd_noalloc(x.data_ptr(), gamma.data_ptr(), eps, packed.data_ptr(), scale.data_ptr(),
+                                          M, K, N, y.data_ptr(), _stream(stream)), "mmf_bitlinear_fwd_noalloc")
+    return y
 
 
 def hbm_copy(src: torch.Tensor, dst: torch.Tensor, stream=None):

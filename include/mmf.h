@@ -180,6 +180,41 @@ int mmf_bitlinear_fwd_group(const uint16_t* x, const float* gamma, float eps,
                             unsigned flags, void* stream);
 
 /*
+ * mmf_bitlinear_fwd_noalloc -- mmf_bitlinear_fwd without a caller-supplied
+ * workspace; nothing on the pages corresponds to it (it is an interface
+ * convenience, not part of the method).
+ *
+ * Some callers cannot allocate device memory: a plug-in hosted by another
+ * runtime that owns all device memory through its own pool (a raw cudaMalloc
+ * would bypass that pool's accounting and may fail or fragment it), or a
+ * latency-critical caller that must not block in cudaMalloc / cudaFree, which
+ * can synchronise the device.  This entry point serves them: the caller passes
+ * only inputs and outputs, exactly as for mmf_bitlinear_fwd (same arguments
+ * minus the workspace, same results bit for bit), and the large-M workspace
+ * comes from a static device array inside the library instead.
+ *
+ * Limits and behaviour:
+ *   - The static scratch holds MMF_NOALLOC_SCRATCH_BYTES bytes (64 MiB);
+ *     shapes with mmf_workspace_bytes(M, K, N) above that return
+ *     MMF_ERR_WORKSPACE and launch nothing.  Every GPU that loads the library
+ *     holds the 64 MiB until the process exits.
+ *   - No call allocates or frees device memory.
+ *   - The first call on a device (with a workspace-needing shape) looks up
+ *     the scratch's device address for that device; make that first call
+ *     before any stream capture on the device.
+ *   - All calls on a device share the one scratch array.  Calls whose kernels
+ *     overlap on the GPU (different streams, or threads with their own
+ *     streams) race on it and give wrong results; order them, e.g. on one
+ *     stream.  Nothing in the scratch needs clearing between calls: each call
+ *     rewrites every byte it reads.
+ */
+#define MMF_NOALLOC_SCRATCH_BYTES (64u << 20)
+int mmf_bitlinear_fwd_noalloc(const uint16_t* x, const float* gamma, float eps,
+                              const uint32_t* packed, const float* scale,
+                              int64_t M, int64_t K, int64_t N, uint16_t* y,
+                              void* stream);
+
+/*
  * mmf_hbm_copy -- streaming device-to-device copy of `bytes` bytes (a multiple
  * of 16) with 128-bit loads and stores.  Measurement kernel: it gives the HBM
  * bandwidth the roofline fractions are stated against.  src and dst must not
