@@ -221,6 +221,23 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// AND of a predicate over the `count` threads of named barrier `id` (all of
+// them must call it); every thread gets the same answer, so a group that has
+// to leave a loop together can decide together.
+template <int id, int count>
+__device__ __forceinline__ bool named_barrier_and(bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(out)
+        : "r"(static_cast<uint32_t>(pred)), "n"(id), "n"(count)
+        : "memory");
+    return out != 0;
+}
+
 // ---------------------------------------------------------------------------
 // Programmatic dependent launch
 // ---------------------------------------------------------------------------

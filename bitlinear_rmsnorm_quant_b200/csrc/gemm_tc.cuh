@@ -8,16 +8,20 @@
 // sum_k w~ q = (sum over w~=+1 of q) - (sum over w~=-1 of q)
 // (the ternary accumulation of ld246.com, section "三值权重的应用").
 //
-// Tile: 128 weight rows (MMA M) x BT tokens (MMA N) x 128 K per stage; the
+// Tile: 128 weight rows (MMA M) x BT tokens (MMA N), K in stages of 128; the
 // weights are the A operand, so one unpacked weight tile feeds BT tokens.
-// Warp roles (256 threads):
+// Persistent: one CTA per SM walks the tiles (token tile major, weight tile
+// minor, so CTAs working at the same time share activation tiles in L2), with
+// two TMEM accumulators so a tile's epilogue overlaps the next tile's MMAs.
+// Warp roles (384 threads):
 //   warp 0      TMA producer: q tile (BT x 128 B, 128-byte swizzle) and the
 //               packed weight tile (128 x 32 B) per stage
 //   warp 1      TMEM allocation; lane 0 issues tcgen05.mma (4 x K=32 per
-//               stage) and tcgen05.commit
-//   warps 4-7   unpack: thread u expands row u's 128 codes to int8 in the
-//               128-byte-swizzled K-major layout the MMA reads; then the
-//               epilogue (tcgen05.ld, subtract qsum, rescale, store)
+//               stage) and the tcgen05.commits
+//   warps 4-7   epilogue: tcgen05.ld, subtract sum q, rescale, transpose
+//               through shared memory, 16-byte stores of y
+//   warps 8-11  unpack: thread u expands row u's 128 codes to int8 in the
+//               128-byte-swizzled K-major layout the MMA reads
 // Every wait is bounded; on timeout the CTA records the error, drains its
 // copies and MMAs, frees TMEM and exits.
 #pragma once
@@ -28,26 +32,30 @@ namespace mmf {
 constexpr int kTcRows = 128;      // weight rows per tile (MMA M)
 constexpr int kTcK = 128;         // K (bytes of int8) per stage
 constexpr int kTcStages = 4;
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 384;
 constexpr int kTcPackedBytes = kTcRows * (kTcK / 4);  // 4 KB of 2-bit codes per stage
+constexpr int kTcEpiBarrier = 2;                       // named barrier of the epilogue warps
 
 template <int BT>
 struct TcLayout {
     static constexpr int a_bytes = kTcRows * kTcK;  // 16 KB
     static constexpr int b_bytes = BT * kTcK;
     static constexpr int stage_bytes = a_bytes + b_bytes + kTcPackedBytes;
-    static constexpr int smem_bytes = kTcStages * stage_bytes + 1024;  // + alignment slack
-    static constexpr int tmem_cols = BT < 32 ? 32 : BT;
+    static constexpr int epi_bytes = 4 * 32 * 32 * 2;  // per-warp 32 x 32 bf16 transpose tiles
+    static constexpr int smem_bytes = kTcStages * stage_bytes + epi_bytes + 1024;  // + alignment slack
+    static constexpr int acc_cols = BT < 32 ? 32 : BT;
+    static constexpr int tmem_cols = 2 * acc_cols;  // double-buffered accumulator
 };
 
 struct TcParams {
-    const int8_t* q;        // unused by the kernel body (read through the tensor map)
     const int* qsum;        // [M]
     const float* absmax;    // [M]      (fused mode)
     const float* scale;     // beta     (fused mode)
     uint16_t* y;            // bf16 [M][N]
     int32_t* acc;           // int32 [M][N]
     int M, K, N;
+    int n_tiles;            // ceil(N / 128)
+    int num_tiles;          // n_tiles * ceil(M / BT)
 };
 
 template <int BT, bool FUSED>
@@ -59,7 +67,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __shared__ __align__(8) uint64_t full_bar[kTcStages];
     __shared__ __align__(8) uint64_t unpacked_bar[kTcStages];
     __shared__ __align__(8) uint64_t empty_bar[kTcStages];
-    __shared__ __align__(8) uint64_t accfull_bar;
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
     __shared__ __align__(8) uint64_t drain_bar;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_flag;
@@ -71,11 +80,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     auto a_tile = [&](int s) { return smem + s * L::stage_bytes; };
     auto b_tile = [&](int s) { return smem + s * L::stage_bytes + L::a_bytes; };
     auto p_tile = [&](int s) { return smem + s * L::stage_bytes + L::a_bytes + L::b_bytes; };
+    uint16_t* epi_tile = reinterpret_cast<uint16_t*>(smem + kTcStages * L::stage_bytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * kTcRows;
-    const int t0 = blockIdx.y * BT;
     const int nk = p.K / kTcK;
+    const int G = gridDim.x;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kTcStages; ++s) {
@@ -83,7 +92,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&unpacked_bar[s], 128);
             mbar_init(&empty_bar[s], 1);
         }
-        mbar_init(&accfull_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull_bar[b], 1);
+            mbar_init(&tempty_bar[b], 4);
+        }
         mbar_init(&drain_bar, 1);
         abort_flag = 0;
         mbar_fence_init();
@@ -98,117 +110,172 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // launched as a programmatic dependent)
     pdl_wait();
     pdl_launch_dependents();
-    if (warp >= 4) {
-        // per-token epilogue constants of this tile
-        for (int i = threadIdx.x - 128; i < BT; i += 128) {
-            const int t = t0 + i;
-            int qs = 0;
-            float cm = 0.0f;
-            if (t < p.M) {
-                qs = p.qsum[t];
-                if constexpr (FUSED) cm = __fmul_rn(__fdiv_rn(p.absmax[t], 127.0f), __ldg(p.scale));
-            }
-            qsum_s[i] = qs;
-            cm_s[i] = cm;
-        }
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_acc = tmem_base_s;
+    const uint32_t tmem_base = tmem_base_s;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int issued = 0;
-            for (int ks = 0; ks < nk; ++ks) {
-                const int s = ks % kTcStages;
-                if (ks >= kTcStages && !mbar_wait(&empty_bar[s], ((ks / kTcStages) - 1) & 1, &abort_flag)) break;
-                mbar_arrive_expect_tx(&full_bar[s], L::b_bytes + kTcPackedBytes);
-                tma_load_2d(b_tile(s), &tmap_q, ks * kTcK, t0, &full_bar[s]);
-                tma_load_2d(p_tile(s), &tmap_w, ks * (kTcK / 4), n0, &full_bar[s]);
-                ++issued;
+            int g = 0;  // stage uses so far
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += G) {
+                const int n0 = (tile % p.n_tiles) * kTcRows;
+                const int t0 = (tile / p.n_tiles) * BT;
+                for (int ks = 0; ks < nk; ++ks, ++g) {
+                    const int s = g % kTcStages;
+                    if (g >= kTcStages && !mbar_wait(&empty_bar[s], ((g / kTcStages) - 1) & 1, &abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full_bar[s], L::b_bytes + kTcPackedBytes);
+                    tma_load_2d(b_tile(s), &tmap_q, ks * kTcK, t0, &full_bar[s]);
+                    tma_load_2d(p_tile(s), &tmap_w, ks * (kTcK / 4), n0, &full_bar[s]);
+                }
             }
+            // Let every copy this CTA started land before the CTA can exit.
             int zero = 0;
-            for (int ks = max(0, issued - kTcStages); ks < issued; ++ks)
-                mbar_wait(&full_bar[ks % kTcStages], (ks / kTcStages) & 1, &zero);
+            for (int u = max(0, g - kTcStages); u < g; ++u)
+                mbar_wait(&full_bar[u % kTcStages], (u / kTcStages) & 1, &zero);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_i8(kTcRows, BT);
-            bool issued_any = false;
-            for (int ks = 0; ks < nk; ++ks) {
-                const int s = ks % kTcStages;
-                const uint32_t par = (ks / kTcStages) & 1;
-                if (!mbar_wait(&full_bar[s], par, &abort_flag)) break;
-                if (!mbar_wait(&unpacked_bar[s], par, &abort_flag)) break;
+            bool issued_any = false, ok = true;
+            int g = 0, li = 0;
+            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += G, ++li) {
+                const int buf = li & 1;
+                if (li >= 2 && !mbar_wait(&tempty_bar[buf], ((li >> 1) - 1) & 1, &abort_flag)) break;
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(a_tile(s)), b0 = smem_u32(b_tile(s));
+                const uint32_t d = tmem_base + static_cast<uint32_t>(buf * L::acc_cols);
+                for (int ks = 0; ks < nk; ++ks, ++g) {
+                    const int s = g % kTcStages;
+                    const uint32_t par = (g / kTcStages) & 1;
+                    if (!mbar_wait(&full_bar[s], par, &abort_flag) || !mbar_wait(&unpacked_bar[s], par, &abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(a_tile(s)), b0 = smem_u32(b_tile(s));
 #pragma unroll
-                for (int kk = 0; kk < kTcK / 32; ++kk) {
-                    mma_i8(tmem_acc, sw128_kmajor_desc(a0 + 32 * kk), sw128_kmajor_desc(b0 + 32 * kk), idesc,
-                           (ks | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < kTcK / 32; ++kk)
+                        mma_i8(d, sw128_kmajor_desc(a0 + 32 * kk), sw128_kmajor_desc(b0 + 32 * kk), idesc,
+                               (ks | kk) != 0 ? 1u : 0u);
+                    issued_any = true;
+                    mma_commit(&empty_bar[s]);
                 }
-                issued_any = true;
-                mma_commit(&empty_bar[s]);
+                if (ok) mma_commit(&tfull_bar[buf]);
             }
-            if (!abort_flag) mma_commit(&accfull_bar);
             if (issued_any) {
                 mma_commit(&drain_bar);
                 int zero = 0;
                 mbar_wait(&drain_bar, 0, &zero);
             }
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 8) {
         // ------------------------------------------------------------ unpack
-        const int u = threadIdx.x - 128;  // weight row within the tile
-        for (int ks = 0; ks < nk; ++ks) {
-            const int s = ks % kTcStages;
-            if (!mbar_wait(&full_bar[s], (ks / kTcStages) & 1, &abort_flag)) break;
-            const uint4* prow = reinterpret_cast<const uint4*>(p_tile(s) + u * (kTcK / 4));
-            const uint4 pa = prow[0], pb = prow[1];
-            const uint32_t words[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-            uint8_t* arow = a_tile(s) + (u >> 3) * 1024 + (u & 7) * 128;
+        const int u = threadIdx.x - 256;  // weight row within the tile
+        int g = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += G) {
+            for (int ks = 0; ks < nk; ++ks, ++g) {
+                const int s = g % kTcStages;
+                if (!mbar_wait(&full_bar[s], (g / kTcStages) & 1, &abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint4* prow = reinterpret_cast<const uint4*>(p_tile(s) + u * (kTcK / 4));
+                const uint4 pa = prow[0], pb = prow[1];
+                const uint32_t words[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+                uint8_t* arow = a_tile(s) + (u >> 3) * 1024 + (u & 7) * 128;
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                // word t holds K bytes 16t .. 16t+15 of this stage; byte-lane j of
-                // the output chunk gets codes 4j .. 4j+3 (bits 2j of each byte)
-                const uint32_t w = words[t];
-                uint4 o;
-                o.x = w & 0x03030303u;
-                o.y = (w >> 2) & 0x03030303u;
-                o.z = (w >> 4) & 0x03030303u;
-                o.w = (w >> 6) & 0x03030303u;
-                *reinterpret_cast<uint4*>(arow + ((t ^ (u & 7)) << 4)) = o;
+                for (int t = 0; t < 8; ++t) {
+                    // word t holds K bytes 16t .. 16t+15 of this stage; byte-lane j of
+                    // the output chunk gets codes 4j .. 4j+3 (bits 2j of each byte)
+                    const uint32_t w = words[t];
+                    uint4 o;
+                    o.x = w & 0x03030303u;
+                    o.y = (w >> 2) & 0x03030303u;
+                    o.z = (w >> 4) & 0x03030303u;
+                    o.w = (w >> 6) & 0x03030303u;
+                    *reinterpret_cast<uint4*>(arow + ((t ^ (u & 7)) << 4)) = o;
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&unpacked_bar[s]);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(&unpacked_bar[s]);
         }
-
+    } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue
-        const int wq = warp - 4;  // TMEM lanes 32*wq .. 32*wq+31
-        const int n = n0 + 32 * wq + lane;
-        const bool ok = mbar_wait(&accfull_bar, 0, &abort_flag);
-        tc_fence_after();
-        if (ok) {
+        const int wq = warp - 4;                    // TMEM lanes 32*wq .. 32*wq+31
+        const int et = threadIdx.x - 128;           // 0..127
+        uint16_t* stg = epi_tile + wq * (32 * 32);  // [32 tokens][32 rows] bf16
+        const bool vec_ok = FUSED && (p.N % 8) == 0;
+        int li = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += G, ++li) {
+            const int buf = li & 1;
+            const int n0 = (tile % p.n_tiles) * kTcRows;
+            const int t0 = (tile / p.n_tiles) * BT;
+            // per-token constants of this tile (the previous tile's are no longer read)
+            asm volatile("bar.sync %0, 128;" ::"n"(kTcEpiBarrier) : "memory");
+            for (int i = et; i < BT; i += 128) {
+                const int t = t0 + i;
+                int qs = 0;
+                float cm = 0.0f;
+                if (t < p.M) {
+                    qs = p.qsum[t];
+                    if constexpr (FUSED) cm = __fmul_rn(__fdiv_rn(p.absmax[t], 127.0f), __ldg(p.scale));
+                }
+                qsum_s[i] = qs;
+                cm_s[i] = cm;
+            }
+            // the four warps leave together or not at all (they share named barriers)
+            const bool got = mbar_wait(&tfull_bar[buf], (li >> 1) & 1, &abort_flag);
+            if (!named_barrier_and<kTcEpiBarrier, 128>(got)) break;
+            tc_fence_after();
+            const int n = n0 + 32 * wq + lane;
+            constexpr int kChunks = BT < 32 ? 1 : BT / 32;
+            constexpr int kCols = BT < 32 ? BT : 32;
 #pragma unroll 1
-            for (int cc = 0; cc < BT / 32 || (BT < 32 && cc == 0); ++cc) {
+            for (int cc = 0; cc < kChunks; ++cc) {
                 uint32_t r[32];
-                const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(32 * wq) << 16) + 32 * cc;
+                const uint32_t taddr = tmem_base + static_cast<uint32_t>(buf * L::acc_cols) +
+                                       (static_cast<uint32_t>(32 * wq) << 16) + 32 * cc;
                 tmem_ld_32x32b_x32(taddr, r);
                 tmem_ld_wait();
-                if (n < p.N) {
-                    const int ncols = BT < 32 ? BT : 32;
+                if (vec_ok) {
+                    // values to the transpose tile: token i, row lane
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        if (i >= ncols) break;
+                    for (int i = 0; i < kCols; ++i) {
+                        const int ti = 32 * cc + i;
+                        const int v = static_cast<int>(r[i]) - qsum_s[ti];
+                        const __nv_bfloat16 yb = __float2bfloat16_rn(__fmul_rn(static_cast<float>(v), cm_s[ti]));
+                        stg[i * 32 + lane] = __bfloat16_as_ushort(yb);
+                    }
+                    __syncwarp();
+                    // 8 rows (16 bytes) per lane: lane covers token lane/4 + 8j, rows 8*(lane%4) ..
+#pragma unroll
+                    for (int j = 0; j < kCols / 8; ++j) {
+                        const int i = (lane >> 2) + 8 * j;
+                        const int t = t0 + 32 * cc + i;
+                        const int nr = n0 + 32 * wq + 8 * (lane & 3);
+                        if (t < p.M && nr < p.N) {
+                            const uint4 v = *reinterpret_cast<const uint4*>(stg + i * 32 + 8 * (lane & 3));
+                            *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(t) * p.N + nr) = v;
+                        }
+                    }
+                    __syncwarp();
+                } else if (n < p.N) {
+#pragma unroll
+                    for (int i = 0; i < kCols; ++i) {
                         const int ti = 32 * cc + i;
                         const int t = t0 + ti;
                         if (t < p.M) {
                             const int v = static_cast<int>(r[i]) - qsum_s[ti];
                             if constexpr (FUSED) {
-                                const __nv_bfloat16 yb = __float2bfloat16_rn(__fmul_rn(static_cast<float>(v), cm_s[ti]));
+                                const __nv_bfloat16 yb =
+                                    __float2bfloat16_rn(__fmul_rn(static_cast<float>(v), cm_s[ti]));
                                 p.y[static_cast<size_t>(t) * p.N + n] = __bfloat16_as_ushort(yb);
                             } else {
                                 p.acc[static_cast<size_t>(t) * p.N + n] = v;
@@ -217,6 +284,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                 }
             }
+            // this accumulator may be overwritten by the tile after next
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[buf]);
         }
     }
 
@@ -224,7 +295,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_acc, L::tmem_cols);
+        tmem_dealloc(tmem_base, L::tmem_cols);
     }
 }
 

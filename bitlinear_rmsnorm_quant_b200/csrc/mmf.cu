@@ -195,25 +195,27 @@ mmf_status make_maps(const int8_t* q, const uint32_t* packed, int64_t M, int64_t
 }
 
 template <int BT>
-mmf_status launch_tc_bt(bool fused, const CUtensorMap& mq, const CUtensorMap& mw, const TcParams& p,
-                        cudaStream_t s, bool pdl) {
-    const dim3 grid(static_cast<unsigned>((p.N + kTcRows - 1) / kTcRows), static_cast<unsigned>((p.M + BT - 1) / BT));
+mmf_status launch_tc_bt(bool fused, const CUtensorMap& mq, const CUtensorMap& mw, TcParams p, cudaStream_t s,
+                        bool pdl, int num_sms) {
+    p.n_tiles = (p.N + kTcRows - 1) / kTcRows;
+    p.num_tiles = p.n_tiles * ((p.M + BT - 1) / BT);
+    const dim3 grid(static_cast<unsigned>(p.num_tiles < num_sms ? p.num_tiles : num_sms));  // persistent
     if (fused) return launch(gemm_tc_kernel<BT, true>, grid, dim3(kTcThreads), TcLayout<BT>::smem_bytes, s, pdl, mq, mw, p);
     return launch(gemm_tc_kernel<BT, false>, grid, dim3(kTcThreads), TcLayout<BT>::smem_bytes, s, pdl, mq, mw, p);
 }
 
 mmf_status launch_tc(bool fused, const int8_t* q, const uint32_t* packed, const TcParams& p, cudaStream_t s,
-                     bool pdl) {
+                     bool pdl, int num_sms) {
     const int BT = token_tile(p.M);
     CUtensorMap mq, mw;
     mmf_status st = make_maps(q, packed, p.M, p.K, p.N, BT, &mq, &mw);
     if (st != MMF_OK) return st;
     switch (BT) {
-        case 16: return launch_tc_bt<16>(fused, mq, mw, p, s, pdl);
-        case 32: return launch_tc_bt<32>(fused, mq, mw, p, s, pdl);
-        case 64: return launch_tc_bt<64>(fused, mq, mw, p, s, pdl);
-        case 128: return launch_tc_bt<128>(fused, mq, mw, p, s, pdl);
-        default: return launch_tc_bt<256>(fused, mq, mw, p, s, pdl);
+        case 16: return launch_tc_bt<16>(fused, mq, mw, p, s, pdl, num_sms);
+        case 32: return launch_tc_bt<32>(fused, mq, mw, p, s, pdl, num_sms);
+        case 64: return launch_tc_bt<64>(fused, mq, mw, p, s, pdl, num_sms);
+        case 128: return launch_tc_bt<128>(fused, mq, mw, p, s, pdl, num_sms);
+        default: return launch_tc_bt<256>(fused, mq, mw, p, s, pdl, num_sms);
     }
 }
 
@@ -291,7 +293,7 @@ mmf_status fwd_impl(const uint16_t* x, const float* gamma, float eps, int64_t M,
         p.N = static_cast<int>(proj[i].N);
         // only the quantiser may overlap the kernel before it: the contraction
         // reads the codes the quantiser writes, and waits for it either way
-        if ((st = launch_tc(true, w.q, proj[i].packed, p, s, pdl)) != MMF_OK) return st;
+        if ((st = launch_tc(true, w.q, proj[i].packed, p, s, pdl, dev->num_sms)) != MMF_OK) return st;
     }
     return MMF_OK;
 }
@@ -407,7 +409,7 @@ int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t 
     p.M = static_cast<int>(M);
     p.K = static_cast<int>(K);
     p.N = static_cast<int>(N);
-    return launch_tc(false, q, packed, p, s, false);
+    return launch_tc(false, q, packed, p, s, false, dev->num_sms);
 }
 
 int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps, const uint32_t* packed, const float* scale,
