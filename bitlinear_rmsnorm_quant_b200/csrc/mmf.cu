@@ -89,7 +89,9 @@ mmf_status device_state(DeviceState** out) {
         if (e == cudaSuccess) e = set_gemv_attrs<6>();
         if (e == cudaSuccess) e = set_gemv_attrs<7>();
         if (e == cudaSuccess) e = set_gemv_attrs<8>();
-        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel, 2 * kMaxK);
+        // up to max(kQuantSmemBudget, one row of the largest K)
+        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<1>, 2 * kMaxK);
+        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8>, 2 * kMaxK);
         if (e != cudaSuccess) return MMF_ERR_CUDA;
         if (!g_encode_tiled) {
             void* fn = nullptr;
@@ -240,9 +242,14 @@ mmf_status launch_gemv(const GemvParams& p, const GemvPlan& plan, cudaStream_t s
 
 mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K, int8_t* q,
                         float* absmax, int* qsum, cudaStream_t s, bool pdl) {
-    const size_t smem = static_cast<size_t>(K) * 2;
-    return launch(rmsnorm_quant_kernel, dim3(static_cast<unsigned>(M)), dim3(kQuantThreads), smem, s, pdl, x, gamma,
-                  eps, static_cast<int>(K), q, absmax, qsum);
+    if (M < kQuantWarpRowMinM)  // one CTA of 8 warps per row
+        return launch(rmsnorm_quant_kernel<8>, dim3(static_cast<unsigned>(M)), dim3(256), static_cast<size_t>(K) * 2,
+                      s, pdl, x, gamma, eps, static_cast<int>(K), M, q, absmax, qsum);
+    const int rows = quant_rows_per_cta(static_cast<int>(K));  // one warp per row
+    const size_t smem = static_cast<size_t>(rows) * K * 2;
+    const int64_t grid = (M + rows - 1) / rows;
+    return launch(rmsnorm_quant_kernel<1>, dim3(static_cast<unsigned>(grid)), dim3(rows * 32), smem, s, pdl, x, gamma,
+                  eps, static_cast<int>(K), M, q, absmax, qsum);
 }
 
 // The fused forward of `count` projections that share x.  Arguments checked.

@@ -3,8 +3,8 @@
 // item "RMS norm"; fused so x is read from HBM once: ld246.com, section
 // "融合 BitLinear 层的创新").
 //
-// One CTA per token row.  The row is streamed from HBM once into shared memory
-// (16-byte loads), then:
+// One warp per token row.  The row is copied from HBM once into shared
+// memory, then:
 //   ms  = (float)(sum x^2 / K)         fp64 sum (bf16 squares are exact in fp64)
 //   inv = 1 / sqrt(ms + eps)           fp32, correctly rounded
 //   r   = (x * inv) * gamma            fp32, two roundings
@@ -58,52 +58,121 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& v, float (&f)[8]) {
     }
 }
 
-__global__ void __launch_bounds__(kQuantThreads) rmsnorm_quant_kernel(const uint16_t* __restrict__ x,
-                                                                      const float* __restrict__ gamma, float eps,
-                                                                      int K, int8_t* __restrict__ q,
-                                                                      float* __restrict__ absmax,
-                                                                      int* __restrict__ qsum) {
-    extern __shared__ uint4 xs[];  // K/8 chunks of 8 bf16
-    __shared__ double red_d[kQuantThreads / 32 + 1];
-    __shared__ float red_f[kQuantThreads / 32 + 1];
-    __shared__ int red_i[kQuantThreads / 32 + 1];
+// WPR warps per token row; a CTA holds kQuantRowsPerCta rows when WPR == 1,
+// else one row.  One thread brings the whole row into shared memory with bulk
+// copies (one request per row, so the row's HBM latency is paid once, not once
+// per 16-byte load); the three passes then run from shared memory.  With one
+// warp per row there is no CTA-wide barrier, so the rows of a CTA proceed
+// independently and the staged bytes per CTA are capped so that at least two
+// CTAs fit on an SM at any K; that form is for large M.  Small M takes 8 warps
+// per row to spread the arithmetic over more SMs.
+constexpr int kQuantRowsPerCta = 8;
+constexpr int kQuantSmemBudget = 112 * 1024;
+constexpr uint32_t kQuantPieceBytes = 32 * 1024;  // bytes per bulk copy request
+constexpr int64_t kQuantWarpRowMinM = 4096;       // rows from which one warp per row pays
 
+__host__ __device__ inline int quant_rows_per_cta(int K) {
+    int r = kQuantSmemBudget / (2 * K);
+    if (r > kQuantRowsPerCta) r = kQuantRowsPerCta;
+    if (r < 1) r = 1;
+    return r;
+}
+
+template <int WPR>
+__global__ void __launch_bounds__(kQuantRowsPerCta * 32) rmsnorm_quant_kernel(const uint16_t* __restrict__ x,
+                                                                              const float* __restrict__ gamma,
+                                                                              float eps, int K, int64_t M,
+                                                                              int8_t* __restrict__ q,
+                                                                              float* __restrict__ absmax,
+                                                                              int* __restrict__ qsum) {
+    extern __shared__ __align__(128) uint4 xs_all[];  // one slice of K/8 chunks per row
+    __shared__ __align__(8) uint64_t row_bar[kQuantRowsPerCta];
+    __shared__ double red_d[WPR];
+    __shared__ float red_f[WPR];
+    __shared__ int red_i[WPR];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rows = (blockDim.x >> 5) / WPR;
+    const int rw = warp / WPR;  // row slot in the CTA
+    const int wr = warp % WPR;  // warp within the row
+    const int64_t m = static_cast<int64_t>(blockIdx.x) * rows + rw;
+    if (wr == 0 && lane == 0) {
+        mbar_init(&row_bar[rw], 1);
+        mbar_fence_init();
+    }
+    if constexpr (WPR == 1) __syncwarp();
+    else __syncthreads();
     pdl_wait();  // x may come from the previous kernel (no-op unless launched as a dependent)
     pdl_launch_dependents();
-    const int64_t m = blockIdx.x;
+    if (m >= M) return;  // WPR == 1: the whole warp; WPR > 1: never (grid = M)
     const int C = K >> 3;
-    const uint4* xr = reinterpret_cast<const uint4*>(x + m * static_cast<int64_t>(K));
-    const float4* g4 = reinterpret_cast<const float4*>(gamma);
-
-    double s2 = 0.0;
-    for (int c = threadIdx.x; c < C; c += kQuantThreads) {
-        const uint4 v = __ldcs(xr + c);  // streamed once: evict-first
-        xs[c] = v;
-        float f[8];
-        unpack_bf16x8(v, f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) s2 += static_cast<double>(f[i]) * static_cast<double>(f[i]);
+    uint4* xs = xs_all + static_cast<size_t>(rw) * C;
+    const uint8_t* xr = reinterpret_cast<const uint8_t*>(x + m * static_cast<int64_t>(K));
+    const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
+    if (wr == 0 && lane == 0) {
+        mbar_arrive_expect_tx(&row_bar[rw], row_bytes);
+        for (uint32_t off = 0; off < row_bytes; off += kQuantPieceBytes) {
+            const uint32_t n = row_bytes - off < kQuantPieceBytes ? row_bytes - off : kQuantPieceBytes;
+            bulk_g2s(reinterpret_cast<uint8_t*>(xs) + off, xr + off, n, &row_bar[rw]);
+        }
     }
-    s2 = block_allreduce(s2, red_d, AddOp());
-    const float ms = static_cast<float>(s2 / static_cast<double>(K));
+    int abort_flag = 0;
+    bool ok = mbar_wait(&row_bar[rw], 0, &abort_flag);
+    if constexpr (WPR == 1) ok = __all_sync(0xffffffffu, ok);
+    else ok = __syncthreads_and(ok);
+    if (!ok) {
+        int no_abort = 0;  // the copy may still be landing in this CTA's shared memory
+        mbar_wait(&row_bar[rw], 0, &no_abort);
+        return;
+    }
+    const float4* g4 = reinterpret_cast<const float4*>(gamma);
+    const int c0 = wr * 32 + lane;
+    constexpr int cstep = WPR * 32;
+
+    // sum x^2: four fp64 chains per thread, a warp tree, then the row's warps in
+    // index order (bf16 squares are exact in fp64)
+    double s2[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int c = c0; c < C; c += cstep) {
+        float f[8];
+        unpack_bf16x8(xs[c], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s2[i & 3] += static_cast<double>(f[i]) * static_cast<double>(f[i]);
+    }
+    double s2w = warp_sum_f64((s2[0] + s2[1]) + (s2[2] + s2[3]));
+    if constexpr (WPR > 1) {
+        if (lane == 0) red_d[wr] = s2w;
+        __syncthreads();
+        s2w = red_d[0];
+#pragma unroll
+        for (int i = 1; i < WPR; ++i) s2w += red_d[i];
+    }
+    const float ms = static_cast<float>(s2w / static_cast<double>(K));
     const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
 
-    float amax = 0.0f;
-    for (int c = threadIdx.x; c < C; c += kQuantThreads) {
+    float amax[2] = {0.0f, 0.0f};
+    for (int c = c0; c < C; c += cstep) {
         float f[8];
         unpack_bf16x8(xs[c], f);
         const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
         const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(f[i], inv), g[i])));
+        for (int i = 0; i < 8; ++i)
+            amax[i & 1] = fmaxf(amax[i & 1], fabsf(__fmul_rn(__fmul_rn(f[i], inv), g[i])));
     }
-    amax = block_allreduce(amax, red_f, MaxOp());
-    const float a = fmaxf(amax, 1e-5f);
+    // amax >= 0, so its bits order like unsigned integers
+    float amax_w = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(amax[0], amax[1]))));
+    if constexpr (WPR > 1) {
+        if (lane == 0) red_f[wr] = amax_w;
+        __syncthreads();
+        amax_w = red_f[0];
+#pragma unroll
+        for (int i = 1; i < WPR; ++i) amax_w = fmaxf(amax_w, red_f[i]);
+    }
+    const float a = fmaxf(amax_w, 1e-5f);
     const float s = __fdiv_rn(127.0f, a);
 
     int qs = 0;
     uint2* qr = reinterpret_cast<uint2*>(q + m * static_cast<int64_t>(K));
-    for (int c = threadIdx.x; c < C; c += kQuantThreads) {
+    for (int c = c0; c < C; c += cstep) {
         float f[8];
         unpack_bf16x8(xs[c], f);
         const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
@@ -117,8 +186,15 @@ __global__ void __launch_bounds__(kQuantThreads) rmsnorm_quant_kernel(const uint
         }
         __stcs(qr + c, make_uint2(packed[0], packed[1]));
     }
-    qs = block_allreduce(qs, red_i, AddOp());
-    if (threadIdx.x == 0) {
+    qs = __reduce_add_sync(0xffffffffu, qs);
+    if constexpr (WPR > 1) {
+        if (lane == 0) red_i[wr] = qs;
+        __syncthreads();
+        qs = red_i[0];
+#pragma unroll
+        for (int i = 1; i < WPR; ++i) qs += red_i[i];
+    }
+    if (wr == 0 && lane == 0) {
         absmax[m] = a;
         if (qsum) qsum[m] = qs;
     }

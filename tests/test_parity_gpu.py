@@ -280,6 +280,32 @@ def test_group_pdl_chain_matches_plain():
         assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("M", [1, 3, 8, 64])
+def test_pdl_dependent_chain(M):
+    """Each call's x is the previous call's y: under PDL the kernels fetch weights
+    before the previous kernel ends but must read x only after it; the chain gives
+    the same bits as ordinary launches."""
+    K = 2048
+    x, g, _ = make_layer(16, M, K, 1)
+    weights = []
+    for i in range(8):
+        W = make_layer(16, 1, K, K, index=i + 1)[2]
+        pk, sc = _pack(W)
+        weights.append((pk, sc, K))
+    gd = g.to(DEV)
+    outs = {}
+    for flags in (0, mmf.FWD_PDL):
+        cur = x.to(DEV)
+        trail = []
+        for w in weights:
+            cur = mmf.bitlinear_fwd_group(cur, gd, [w], EPS, flags=flags)[0]
+            trail.append(cur)
+        torch.cuda.synchronize()
+        outs[flags] = trail
+    for a, b in zip(outs[0], outs[mmf.FWD_PDL]):
+        assert torch.equal(a, b)
+
+
 # -- error paths on the device -----------------------------------------------------------------
 
 def test_argument_errors_on_device():
