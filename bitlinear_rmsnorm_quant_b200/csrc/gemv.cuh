@@ -15,7 +15,7 @@
 // power-of-four lanes are shifted back and summed once per row, and the
 // per-token sum_k q_k is subtracted once.  All integer, exact.
 //
-// CTA: 16 compute warps (8 when M > 4) + 1 producer warp.  The group's weight rows form one
+// CTA: 8 compute warps + 1 producer warp.  The group's weight rows form one
 // concatenated row space; each CTA owns a contiguous range of it.  The
 // producer bulk-copies (TMA) the CTA's weight rows into a ring of small
 // shared-memory stages and gamma into shared memory, then waits for the
@@ -34,10 +34,14 @@ namespace mmf {
 
 constexpr int kGemvMaxComputeWarps = 16;
 
-// compute warps per CTA: 16 while the accumulators are few enough for the
-// register file (M <= 4), else 8; plus one producer warp
-__host__ __device__ constexpr int gemv_compute_warps(int M) { return M <= 4 ? 16 : 8; }
+// 8 compute warps + 1 producer warp.  Up to 4 tokens the registers of two
+// CTAs fit in one SM, so under programmatic dependent launch a CTA of the
+// next kernel can sit beside a running one and stream its weights into shared
+// memory while the running one computes; beyond 4 tokens the accumulators
+// take the register file and one CTA fits.
+__host__ __device__ constexpr int gemv_compute_warps(int) { return 8; }
 __host__ __device__ constexpr int gemv_threads(int M) { return (gemv_compute_warps(M) + 1) * 32; }
+__host__ __device__ constexpr int gemv_ctas_per_sm(int M) { return M <= 4 ? 2 : 1; }
 constexpr int kGemvMaxStages = 8;
 constexpr int kGemvMaxTokens = 8;
 constexpr int kGemvMaxProj = 8;
@@ -137,9 +141,8 @@ __device__ __forceinline__ int gemv_proj_of(const GemvParams& p, int r) {
     return g;
 }
 
-// One CTA per SM: the register file goes to independent accumulator chains.
 template <int MT, bool FUSED>
-__global__ void __launch_bounds__(gemv_threads(MT), 1) gemv_kernel(const __grid_constant__ GemvParams p) {
+__global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_kernel(const __grid_constant__ GemvParams p) {
     constexpr int NW = gemv_compute_warps(MT);
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t full_bar[kGemvMaxStages];

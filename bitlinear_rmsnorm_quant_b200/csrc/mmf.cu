@@ -60,6 +60,14 @@ template <int MT>
 cudaError_t set_gemv_attrs() {
     cudaError_t e = set_smem(gemv_kernel<MT, true>, kGemvSmemBudget);
     if (e == cudaSuccess) e = set_smem(gemv_kernel<MT, false>, kGemvSmemBudget);
+    // All of the SM's unified memory as shared memory: a CTA of the next kernel
+    // can then join a running one without the SM first draining to change the
+    // split between L1 and shared memory (these kernels stage everything they
+    // read in shared memory).
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(gemv_kernel<MT, true>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(gemv_kernel<MT, false>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     return e;
 }
 
