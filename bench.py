@@ -42,6 +42,14 @@ from bitlinear_rmsnorm_quant_b200 import inputs as I  # noqa: E402
 from bitlinear_rmsnorm_quant_b200 import workloads as WL  # noqa: E402
 
 METRIC = "fused RMSNorm+BitLinear tokens/s; GB/s or int8 TOPS as % of B200 roofline"
+
+# DRAM bytes (read + write) per launch of the dominant kernel, mean over the
+# launch shapes of one layer set, from the ncu captures summarised in
+# profiles/.  An entry must be removed whenever its kernel changes.
+NCU_TRAFFIC = {
+    "decode-2.7b-m1": {"bytes_per_launch": 6677000, "source": "profiles/gemv_decode-2.7b-m1.md"},
+    "prefill-1.3b": {"bytes_per_launch": 40480000, "source": "profiles/gemm_tc_prefill-1.3b.md"},
+}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 2.0   # nominal dense ratio int8 : bf16 (4.5 : 2.25 POPS)
@@ -331,19 +339,26 @@ def run_ours(args, dist: Dist):
     e2e_value = tokens_per_step / (e2e_ms / 1e3)
 
     peaks, peak_src = load_peaks()
+    traffic = NCU_TRAFFIC.get(wl.name) if args.layers == 0 and args.api == "group" else None
     if decode_path:
         achieved = bytes_per_step / (ms / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": None, "kernel": "gemv_kernel",
+                "frac": round(achieved / peak, 4), "kernel": "gemv_kernel",
+                "traffic": traffic["bytes_per_launch"] if traffic else None,
+                "traffic_source": traffic["source"] if traffic else None,
+                "algorithmic_bytes_per_launch": round(bytes_per_step / launches_per_step),
                 "peak_source": f"{peak_src} hbm_gbs (copy of 1 Gi bf16, read+write bytes)",
                 "algorithmic_bytes_per_step": bytes_per_step,
-                "note": "step time over all launches, inter-kernel gaps included"}
+                "note": "every launch of the step is this kernel: achieved = bytes per launch / "
+                        "(step time / launches), inter-kernel gaps included"}
     else:
         achieved = ops_per_step / (ms / 1e3) / 1e12
         peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None, "kernel": "gemm_tc_kernel",
+                "frac": round(achieved / peak, 4), "kernel": "gemm_tc_kernel",
+                "traffic": traffic["bytes_per_launch"] if traffic else None,
+                "traffic_source": traffic["source"] if traffic else None,
                 "peak_source": f"{peak_src} bf16_tflops x {INT8_PER_BF16} (nominal int8:bf16 dense ratio)",
                 "algorithmic_ops_per_step": ops_per_step,
                 "note": "int8 TOPS over the whole step (quantiser kernel included)"}

@@ -13,14 +13,16 @@
 // Persistent: one CTA per SM walks the tiles (token tile major, weight tile
 // minor, so CTAs working at the same time share activation tiles in L2), with
 // two TMEM accumulators so a tile's epilogue overlaps the next tile's MMAs.
-// Warp roles (384 threads):
+// Warp roles (640 threads):
 //   warp 0      TMA producer: q tile (BT x 128 B, 128-byte swizzle) and the
 //               packed weight tile (128 x 32 B) per stage
 //   warp 1      TMEM allocation; lane 0 issues tcgen05.mma (4 x K=32 per
 //               stage) and the tcgen05.commits
-//   warps 4-7   epilogue: tcgen05.ld, subtract sum q, rescale, transpose
-//               through shared memory, 16-byte stores of y
-//   warps 8-11  unpack: thread u expands row u's 128 codes to int8 in the
+//   warps 4-15  epilogue, three warps per TMEM sub-partition (a warp reaches
+//               the 32 TMEM lanes of sub-partition warp % 4) taking every
+//               third 32-token chunk: tcgen05.ld, subtract sum q, rescale,
+//               transpose through shared memory, 16-byte stores of y
+//   warps 16-19 unpack: thread u expands row u's 128 codes to int8 in the
 //               128-byte-swizzled K-major layout the MMA reads
 // Every wait is bounded; on timeout the CTA records the error, drains its
 // copies and MMAs, frees TMEM and exits.
@@ -32,7 +34,8 @@ namespace mmf {
 constexpr int kTcRows = 128;      // weight rows per tile (MMA M)
 constexpr int kTcK = 128;         // K (bytes of int8) per stage
 constexpr int kTcStages = 4;
-constexpr int kTcThreads = 384;
+constexpr int kTcEpiWarps = 12;                        // three per TMEM sub-partition
+constexpr int kTcThreads = (8 + kTcEpiWarps) * 32;     // warps 0-3 TMA/MMA/idle, epilogue, 4 unpack
 constexpr int kTcPackedBytes = kTcRows * (kTcK / 4);  // 4 KB of 2-bit codes per stage
 constexpr int kTcEpiBarrier = 2;                       // named barrier of the epilogue warps
 
@@ -41,7 +44,7 @@ struct TcLayout {
     static constexpr int a_bytes = kTcRows * kTcK;  // 16 KB
     static constexpr int b_bytes = BT * kTcK;
     static constexpr int stage_bytes = a_bytes + b_bytes + kTcPackedBytes;
-    static constexpr int epi_bytes = 4 * 32 * 32 * 2;  // per-warp 32 x 32 bf16 transpose tiles
+    static constexpr int epi_bytes = kTcEpiWarps * 16 * 32 * 2;  // per-warp 16 x 32 bf16 transpose tiles
     static constexpr int smem_bytes = kTcStages * stage_bytes + epi_bytes + 1024;  // + alignment slack
     static constexpr int acc_cols = BT < 32 ? 32 : BT;
     static constexpr int tmem_cols = 2 * acc_cols;  // double-buffered accumulator
@@ -94,7 +97,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull_bar[b], 1);
-            mbar_init(&tempty_bar[b], 4);
+            mbar_init(&tempty_bar[b], kTcEpiWarps);
         }
         mbar_init(&drain_bar, 1);
         abort_flag = 0;
@@ -174,9 +177,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mbar_wait(&drain_bar, 0, &zero);
             }
         }
-    } else if (warp >= 8) {
+    } else if (warp >= 4 + kTcEpiWarps) {
         // ------------------------------------------------------------ unpack
-        const int u = threadIdx.x - 256;  // weight row within the tile
+        const int u = threadIdx.x - (4 + kTcEpiWarps) * 32;  // weight row within the tile
         int g = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += G) {
@@ -208,9 +211,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue
-        const int wq = warp - 4;                    // TMEM lanes 32*wq .. 32*wq+31
-        const int et = threadIdx.x - 128;           // 0..127
-        uint16_t* stg = epi_tile + wq * (32 * 32);  // [32 tokens][32 rows] bf16
+        const int wq = warp & 3;                    // TMEM lanes 32*wq .. 32*wq+31 (a warp's sub-partition)
+        const int half = (warp - 4) >> 2;           // which of the warps of that sub-partition
+        const int et = threadIdx.x - 128;           // 0 .. 32*kTcEpiWarps-1
+        uint16_t* stg = epi_tile + (warp - 4) * (16 * 32);  // [16 tokens][32 rows] bf16
         const bool vec_ok = FUSED && (p.N % 8) == 0;
         int li = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += G, ++li) {
@@ -218,8 +222,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int n0 = (tile % p.n_tiles) * kTcRows;
             const int t0 = (tile / p.n_tiles) * BT;
             // per-token constants of this tile (the previous tile's are no longer read)
-            asm volatile("bar.sync %0, 128;" ::"n"(kTcEpiBarrier) : "memory");
-            for (int i = et; i < BT; i += 128) {
+            asm volatile("bar.sync %0, %1;" ::"n"(kTcEpiBarrier), "n"(kTcEpiWarps * 32) : "memory");
+            for (int i = et; i < BT; i += kTcEpiWarps * 32) {
                 const int t = t0 + i;
                 int qs = 0;
                 float cm = 0.0f;
@@ -232,40 +236,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             // the four warps leave together or not at all (they share named barriers)
             const bool got = mbar_wait(&tfull_bar[buf], (li >> 1) & 1, &abort_flag);
-            if (!named_barrier_and<kTcEpiBarrier, 128>(got)) break;
+            if (!named_barrier_and<kTcEpiBarrier, kTcEpiWarps * 32>(got)) break;
             tc_fence_after();
             const int n = n0 + 32 * wq + lane;
             constexpr int kChunks = BT < 32 ? 1 : BT / 32;
             constexpr int kCols = BT < 32 ? BT : 32;
 #pragma unroll 1
-            for (int cc = 0; cc < kChunks; ++cc) {
+            for (int cc = half; cc < kChunks; cc += kTcEpiWarps / 4) {
                 uint32_t r[32];
                 const uint32_t taddr = tmem_base + static_cast<uint32_t>(buf * L::acc_cols) +
                                        (static_cast<uint32_t>(32 * wq) << 16) + 32 * cc;
                 tmem_ld_32x32b_x32(taddr, r);
                 tmem_ld_wait();
                 if (vec_ok) {
-                    // values to the transpose tile: token i, row lane
+                    // 16 tokens at a time through the transpose tile: token i, row lane
 #pragma unroll
-                    for (int i = 0; i < kCols; ++i) {
-                        const int ti = 32 * cc + i;
-                        const int v = static_cast<int>(r[i]) - qsum_s[ti];
-                        const __nv_bfloat16 yb = __float2bfloat16_rn(__fmul_rn(static_cast<float>(v), cm_s[ti]));
-                        stg[i * 32 + lane] = __bfloat16_as_ushort(yb);
-                    }
-                    __syncwarp();
-                    // 8 rows (16 bytes) per lane: lane covers token lane/4 + 8j, rows 8*(lane%4) ..
+                    for (int h = 0; h < (kCols + 15) / 16; ++h) {
 #pragma unroll
-                    for (int j = 0; j < kCols / 8; ++j) {
-                        const int i = (lane >> 2) + 8 * j;
-                        const int t = t0 + 32 * cc + i;
-                        const int nr = n0 + 32 * wq + 8 * (lane & 3);
-                        if (t < p.M && nr < p.N) {
-                            const uint4 v = *reinterpret_cast<const uint4*>(stg + i * 32 + 8 * (lane & 3));
-                            *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(t) * p.N + nr) = v;
+                        for (int i = 0; i < 16 && 16 * h + i < kCols; ++i) {
+                            const int ti = 32 * cc + 16 * h + i;
+                            const int v = static_cast<int>(r[16 * h + i]) - qsum_s[ti];
+                            const __nv_bfloat16 yb =
+                                __float2bfloat16_rn(__fmul_rn(static_cast<float>(v), cm_s[ti]));
+                            stg[i * 32 + lane] = __bfloat16_as_ushort(yb);
                         }
+                        __syncwarp();
+                        // 8 rows (16 bytes) per lane: lane covers token lane/4 + 8j, rows 8*(lane%4) ..
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const int i = (lane >> 2) + 8 * j;
+                            const int t = t0 + 32 * cc + 16 * h + i;
+                            const int nr = n0 + 32 * wq + 8 * (lane & 3);
+                            if (16 * h + i < kCols && t < p.M && nr < p.N) {
+                                const uint4 v = *reinterpret_cast<const uint4*>(stg + i * 32 + 8 * (lane & 3));
+                                *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(t) * p.N + nr) = v;
+                            }
+                        }
+                        __syncwarp();
                     }
-                    __syncwarp();
                 } else if (n < p.N) {
 #pragma unroll
                     for (int i = 0; i < kCols; ++i) {

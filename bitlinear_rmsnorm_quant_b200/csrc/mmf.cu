@@ -97,9 +97,8 @@ mmf_status device_state(DeviceState** out) {
         if (e == cudaSuccess) e = set_gemv_attrs<6>();
         if (e == cudaSuccess) e = set_gemv_attrs<7>();
         if (e == cudaSuccess) e = set_gemv_attrs<8>();
-        // up to max(kQuantSmemBudget, one row of the largest K)
-        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<1>, 2 * kMaxK);
-        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8>, 2 * kMaxK);
+        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_stream_kernel, quant_stream_smem(kMaxQuantStreamK));
+        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8>, 2 * kMaxK);  // one row of the largest K
         if (e != cudaSuccess) return MMF_ERR_CUDA;
         if (!g_encode_tiled) {
             void* fn = nullptr;
@@ -249,15 +248,21 @@ mmf_status launch_gemv(const GemvParams& p, const GemvPlan& plan, cudaStream_t s
 }
 
 mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K, int8_t* q,
-                        float* absmax, int* qsum, cudaStream_t s, bool pdl) {
-    if (M < kQuantWarpRowMinM)  // one CTA of 8 warps per row
+                        float* absmax, int* qsum, cudaStream_t s, bool pdl, int num_sms) {
+    if (M < kQuantWarpRowMinM || K > kMaxQuantStreamK)  // one CTA of 8 warps per row
         return launch(rmsnorm_quant_kernel<8>, dim3(static_cast<unsigned>(M)), dim3(256), static_cast<size_t>(K) * 2,
                       s, pdl, x, gamma, eps, static_cast<int>(K), M, q, absmax, qsum);
-    const int rows = quant_rows_per_cta(static_cast<int>(K));  // one warp per row
-    const size_t smem = static_cast<size_t>(rows) * K * 2;
-    const int64_t grid = (M + rows - 1) / rows;
-    return launch(rmsnorm_quant_kernel<1>, dim3(static_cast<unsigned>(grid)), dim3(rows * 32), smem, s, pdl, x, gamma,
-                  eps, static_cast<int>(K), M, q, absmax, qsum);
+    // persistent: as many CTAs as fit on the SMs at once, never more than the rows need
+    const size_t smem = quant_stream_smem(static_cast<int>(K));
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rmsnorm_quant_stream_kernel, kQuantStreamWarps * 32,
+                                                      smem) != cudaSuccess || per_sm < 1)
+        return MMF_ERR_CUDA;
+    int64_t grid = static_cast<int64_t>(per_sm) * num_sms;
+    const int64_t need = (M + kQuantStreamWarps - 1) / kQuantStreamWarps;
+    if (grid > need) grid = need;
+    return launch(rmsnorm_quant_stream_kernel, dim3(static_cast<unsigned>(grid)), dim3(kQuantStreamWarps * 32), smem,
+                  s, pdl, x, gamma, eps, static_cast<int>(K), M, q, absmax, qsum);
 }
 
 // The fused forward of `count` projections that share x.  Arguments checked.
@@ -294,7 +299,7 @@ mmf_status fwd_impl(const uint16_t* x, const float* gamma, float eps, int64_t M,
         return launch_gemv<true>(p, plan, s, pdl);
     }
     Workspace w = carve(workspace, M, K);
-    mmf_status st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s, pdl);
+    mmf_status st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s, pdl, dev->num_sms);
     if (st != MMF_OK) return st;
     for (int i = 0; i < count; ++i) {
         if (proj[i].N == 0) continue;
@@ -381,7 +386,7 @@ int mmf_quantize_act(const uint16_t* x, const float* gamma, float eps, int64_t M
     if (!aligned16(x) || !aligned16(gamma) || !aligned16(q) || !aligned16(absmax)) return MMF_ERR_MISALIGNED;
     DeviceState* dev;
     if ((st = device_state(&dev)) != MMF_OK) return st;
-    return launch_quant(x, gamma, eps, M, K, q, absmax, nullptr, static_cast<cudaStream_t>(stream), false);
+    return launch_quant(x, gamma, eps, M, K, q, absmax, nullptr, static_cast<cudaStream_t>(stream), false, dev->num_sms);
 }
 
 int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t K, int64_t N, int32_t* acc,

@@ -200,6 +200,122 @@ __global__ void __launch_bounds__(kQuantRowsPerCta * 32) rmsnorm_quant_kernel(co
     }
 }
 
+// Large M: a persistent grid; warp w of the grid takes rows w, w + W, w + 2W,
+// ... (W warps in the grid) and double-buffers them, so the bulk copy of its
+// next row is in flight while it works on the current one.  Each row: the sum
+// of squares in fp64 (exact for bf16 squares, so the order of the additions
+// does not matter), the absmax of r = (x * inv) * gamma, then the codes.  A
+// code is rounded by one float addition: in [2^23, 2^24) consecutive floats
+// are 1 apart, so adding 1.5 * 2^23 to v = r * s (|v| <= 127 up to one ulp,
+// since s = 127 / a and a >= |r|) rounds v to the nearest integer, ties to
+// even, and leaves it in the low byte (1.5 * 2^23 has a zero low byte).  The
+// same integer as rint(v), which is already within [-127, 127], so the clamp
+// of the definition never changes a code.  Four bytes are packed with byte
+// permutes and summed with one DP4A.
+constexpr int kQuantStreamWarps = 8;
+constexpr int kMaxQuantStreamK = 7168;  // 8 warps x 2 rows of bf16 within the 227 KB of one CTA
+
+__host__ __device__ inline size_t quant_stream_smem(int K) {
+    return static_cast<size_t>(kQuantStreamWarps) * 2 * 2 * static_cast<size_t>(K);
+}
+
+__global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ gamma, float eps, int K, int64_t M,
+    int8_t* __restrict__ q, float* __restrict__ absmax, int* __restrict__ qsum) {
+    extern __shared__ __align__(128) uint4 xs_all[];  // [warp][2 buffers][K/8 chunks]
+    __shared__ __align__(8) uint64_t row_bar[kQuantStreamWarps][2];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int C = K >> 3;
+    const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * kQuantStreamWarps + warp;
+    const int64_t TW = static_cast<int64_t>(gridDim.x) * kQuantStreamWarps;
+    auto buf = [&](int b) { return xs_all + (static_cast<size_t>(warp) * 2 + b) * C; };
+    if (lane == 0) {
+        mbar_init(&row_bar[warp][0], 1);
+        mbar_init(&row_bar[warp][1], 1);
+        mbar_fence_init();
+    }
+    __syncwarp();
+    pdl_wait();  // x may come from the previous kernel (no-op unless launched as a dependent)
+    pdl_launch_dependents();
+    auto issue = [&](int64_t m, int b) {
+        if (lane == 0) {
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(x + m * static_cast<int64_t>(K));
+            mbar_arrive_expect_tx(&row_bar[warp][b], row_bytes);
+            for (uint32_t off = 0; off < row_bytes; off += kQuantPieceBytes) {
+                const uint32_t n = row_bytes - off < kQuantPieceBytes ? row_bytes - off : kQuantPieceBytes;
+                bulk_g2s(reinterpret_cast<uint8_t*>(buf(b)) + off, src + off, n, &row_bar[warp][b]);
+            }
+        }
+    };
+    if (gw < M) issue(gw, 0);
+    const float4* g4 = reinterpret_cast<const float4*>(gamma);
+    int i = 0;
+    for (int64_t m = gw; m < M; m += TW, ++i) {
+        const int b = i & 1;
+        const bool next = m + TW < M;
+        if (next) issue(m + TW, b ^ 1);  // that buffer's last row was finished in the previous iteration
+        int abort_flag = 0;
+        if (!__all_sync(0xffffffffu, mbar_wait(&row_bar[warp][b], (i >> 1) & 1, &abort_flag))) {
+            int no_abort = 0;  // let the copies in flight land in this CTA's shared memory
+            mbar_wait(&row_bar[warp][b], (i >> 1) & 1, &no_abort);
+            if (next) mbar_wait(&row_bar[warp][b ^ 1], ((i + 1) >> 1) & 1, &no_abort);
+            return;
+        }
+        const uint4* xs = buf(b);
+
+        double s2[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int c = lane; c < C; c += 32) {
+            float f[8];
+            unpack_bf16x8(xs[c], f);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) s2[k & 3] += static_cast<double>(f[k]) * static_cast<double>(f[k]);
+        }
+        const double s2w = warp_sum_f64((s2[0] + s2[1]) + (s2[2] + s2[3]));
+        const float ms = static_cast<float>(s2w / static_cast<double>(K));
+        const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+
+        float amax[2] = {0.0f, 0.0f};
+        for (int c = lane; c < C; c += 32) {
+            float f[8];
+            unpack_bf16x8(xs[c], f);
+            const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
+            const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                amax[k & 1] = fmaxf(amax[k & 1], fabsf(__fmul_rn(__fmul_rn(f[k], inv), g[k])));
+        }
+        // amax >= 0, so its bits order like unsigned integers
+        const float amax_w = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(amax[0], amax[1]))));
+        const float a = fmaxf(amax_w, 1e-5f);
+        const float s = __fdiv_rn(127.0f, a);
+
+        int qs = 0;
+        uint2* qr = reinterpret_cast<uint2*>(q + m * static_cast<int64_t>(K));
+        for (int c = lane; c < C; c += 32) {
+            float f[8];
+            unpack_bf16x8(xs[c], f);
+            const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
+            const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            uint32_t cb[8];  // codes in the low bytes
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                cb[k] = __float_as_uint(__fadd_rn(__fmul_rn(__fmul_rn(__fmul_rn(f[k], inv), g[k]), s), 12582912.0f));
+            const uint32_t w0 = __byte_perm(__byte_perm(cb[0], cb[1], 0x0040), __byte_perm(cb[2], cb[3], 0x0040), 0x5410);
+            const uint32_t w1 = __byte_perm(__byte_perm(cb[4], cb[5], 0x0040), __byte_perm(cb[6], cb[7], 0x0040), 0x5410);
+            qs = __dp4a(static_cast<int>(w0), 0x01010101, qs);
+            qs = __dp4a(static_cast<int>(w1), 0x01010101, qs);
+            __stcs(qr + c, make_uint2(w0, w1));
+        }
+        qs = __reduce_add_sync(0xffffffffu, qs);
+        if (lane == 0) {
+            absmax[m] = a;
+            if (qsum) qsum[m] = qs;
+        }
+        __syncwarp();  // every lane is done with this buffer before it is refilled
+    }
+}
+
 // qsum only (for the contraction alone, when q is given).
 __global__ void __launch_bounds__(kQuantThreads) qsum_kernel(const int8_t* __restrict__ q, int K,
                                                              int* __restrict__ qsum) {

@@ -7,9 +7,10 @@ phần lõi: MLGRU và GLU").  Every input is drawn by ``inputs`` from a seed; n
 dataset is read.
 
 A ``Projection`` is one BitLinear d_in -> d_out.  ``input_index`` names which
-activation tensor feeds it: projections with the same index share one x (the
-MLGRU gates share the token mixer's input, the GLU gate/up share the channel
-mixer's input).
+activation tensor feeds it: projections with the same index share one x.  In
+the token mixer (MLGRU) the f, c and g projections read the mixer's input and
+o reads the gated hidden state g*h, its own input; in the channel mixer (GLU)
+gate and up share the mixer's input and down reads their product.
 """
 from __future__ import annotations
 
@@ -52,9 +53,9 @@ def _set_1p3b():
     d, f = 2048, 5632
     return (
         Projection("f", d, d, 0), Projection("c", d, d, 0),
-        Projection("g", d, d, 0), Projection("o", d, d, 0),
-        Projection("gate", d, f, 1), Projection("up", d, f, 1),
-        Projection("down", f, d, 2),
+        Projection("g", d, d, 0), Projection("o", d, d, 1),
+        Projection("gate", d, f, 2), Projection("up", d, f, 2),
+        Projection("down", f, d, 3),
     )
 
 
@@ -62,9 +63,9 @@ def _set_2p7b():
     d, f = 2560, 6912
     return (
         Projection("f", d, d, 0), Projection("c", d, d, 0),
-        Projection("g", d, d, 0), Projection("o", d, d, 0),
-        Projection("gate", d, f, 1), Projection("up", d, f, 1),
-        Projection("down", f, d, 2),
+        Projection("g", d, d, 0), Projection("o", d, d, 1),
+        Projection("gate", d, f, 2), Projection("up", d, f, 2),
+        Projection("down", f, d, 3),
     )
 
 

@@ -11,6 +11,7 @@ import pytest
 import torch
 
 from bitlinear_rmsnorm_quant_b200 import mmf
+from bitlinear_rmsnorm_quant_b200 import inputs as I
 from bitlinear_rmsnorm_quant_b200 import workloads as WL
 from gpu_cases import (Q_MAX_DIFF_FRAC, Y_REL_TOL, bits_np, make_layer, q_diff_stats, y_rel_error)
 
@@ -79,7 +80,10 @@ def test_pack_special_matrices(oracle):
 # -- RMSNorm + quantisation ------------------------------------------------------------
 
 @pytest.mark.parametrize("M,K,outliers", [(16, 256, 0.0), (5, 128, 0.0), (300, 2048, 0.0), (37, 6912, 0.01),
-                                          (64, 5632, 0.0)])
+                                          (64, 5632, 0.0),
+                                          # large M: the persistent double-buffered quantiser
+                                          (4100, 1024, 0.0), (4096, 7168, 0.01), (5000, 128, 0.0),
+                                          (4097, 7296, 0.0)])
 def test_quantize_act(oracle, M, K, outliers):
     x, g, _ = make_layer(9, M, K, 1, outlier_frac=outliers)
     q, a = mmf.quantize_act(x.to(DEV), g.to(DEV), EPS)
@@ -182,7 +186,8 @@ def test_smoke_config(oracle):
                          ids=lambda w: w.name)
 def test_decode_configs(oracle, wl):
     for j, p in enumerate(wl.projections):
-        x, g, W = make_layer(wl.seed, wl.M, p.K, p.N, index=p.input_index, outlier_frac=wl.outlier_frac)
+        x, g, _ = make_layer(wl.seed, wl.M, p.K, 1, index=p.input_index, outlier_frac=wl.outlier_frac)
+        W = I.latent_weights(wl.seed, p.N, p.K, index=16 + j)  # each projection its own matrix
         _layer_parity(oracle, x, g, W)
 
 
