@@ -75,8 +75,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __shared__ __align__(8) uint64_t drain_bar;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_flag;
-    __shared__ int qsum_s[BT];
-    __shared__ float cm_s[BT];
+    __shared__ __align__(16) int qsum_s[BT < 16 ? 16 : BT];
+    __shared__ __align__(16) float cm_s[BT < 16 ? 16 : BT];
 
     // 1024-byte aligned base (128-byte swizzle atoms are 8 rows x 128 B)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -249,27 +249,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tmem_ld_32x32b_x32(taddr, r);
                 tmem_ld_wait();
                 if (vec_ok) {
-                    // 16 tokens at a time through the transpose tile: token i, row lane
+                    // 16 tokens at a time through the transpose tile, as bf16 pairs:
+                    // word (pair i/2, row lane) holds tokens i and i+1 of this lane's row
+                    uint32_t* stg32 = reinterpret_cast<uint32_t*>(stg);
 #pragma unroll
                     for (int h = 0; h < (kCols + 15) / 16; ++h) {
 #pragma unroll
-                        for (int i = 0; i < 16 && 16 * h + i < kCols; ++i) {
-                            const int ti = 32 * cc + 16 * h + i;
-                            const int v = static_cast<int>(r[16 * h + i]) - qsum_s[ti];
-                            const __nv_bfloat16 yb =
-                                __float2bfloat16_rn(__fmul_rn(static_cast<float>(v), cm_s[ti]));
-                            stg[i * 32 + lane] = __bfloat16_as_ushort(yb);
+                        for (int i8 = 0; i8 < 16 && 16 * h + i8 < kCols; i8 += 8) {
+                            // per-token constants, 8 tokens per pair of broadcast 16-byte loads
+                            const int tb = 32 * cc + 16 * h + i8;
+                            const int4 qa = *reinterpret_cast<const int4*>(qsum_s + tb);
+                            const int4 qb = *reinterpret_cast<const int4*>(qsum_s + tb + 4);
+                            const float4 ca = *reinterpret_cast<const float4*>(cm_s + tb);
+                            const float4 cb = *reinterpret_cast<const float4*>(cm_s + tb + 4);
+                            const int qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+                            const float cv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+                            for (int k = 0; k < 8; k += 2) {
+                                const int v0 = static_cast<int>(r[16 * h + i8 + k]) - qv[k];
+                                const int v1 = static_cast<int>(r[16 * h + i8 + k + 1]) - qv[k + 1];
+                                const __nv_bfloat162 y2 = __floats2bfloat162_rn(__fmul_rn(static_cast<float>(v0), cv[k]),
+                                                                                __fmul_rn(static_cast<float>(v1), cv[k + 1]));
+                                stg32[((i8 + k) >> 1) * 32 + lane] = *reinterpret_cast<const uint32_t*>(&y2);
+                            }
                         }
                         __syncwarp();
-                        // 8 rows (16 bytes) per lane: lane covers token lane/4 + 8j, rows 8*(lane%4) ..
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const int i = (lane >> 2) + 8 * j;
-                            const int t = t0 + 32 * cc + 16 * h + i;
+                        // lane: token pair lane/4, rows 8*(lane%4) .. +7 -> two 16-byte stores
+                        {
+                            const int pr = lane >> 2;
                             const int nr = n0 + 32 * wq + 8 * (lane & 3);
-                            if (16 * h + i < kCols && t < p.M && nr < p.N) {
-                                const uint4 v = *reinterpret_cast<const uint4*>(stg + i * 32 + 8 * (lane & 3));
-                                *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(t) * p.N + nr) = v;
+                            const uint4 wa = *reinterpret_cast<const uint4*>(stg32 + pr * 32 + 8 * (lane & 3));
+                            const uint4 wb = *reinterpret_cast<const uint4*>(stg32 + pr * 32 + 8 * (lane & 3) + 4);
+                            const uint4 even = make_uint4(__byte_perm(wa.x, wa.y, 0x5410), __byte_perm(wa.z, wa.w, 0x5410),
+                                                          __byte_perm(wb.x, wb.y, 0x5410), __byte_perm(wb.z, wb.w, 0x5410));
+                            const uint4 odd = make_uint4(__byte_perm(wa.x, wa.y, 0x7632), __byte_perm(wa.z, wa.w, 0x7632),
+                                                         __byte_perm(wb.x, wb.y, 0x7632), __byte_perm(wb.z, wb.w, 0x7632));
+                            const int i = 16 * h + 2 * pr;
+                            const int t = t0 + 32 * cc + i;
+                            if (i < kCols && nr < p.N) {
+                                if (t < p.M) *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(t) * p.N + nr) = even;
+                                if (t + 1 < p.M) *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(t + 1) * p.N + nr) = odd;
                             }
                         }
                         __syncwarp();
