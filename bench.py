@@ -231,7 +231,12 @@ def run_ours(args, dist: Dist):
     y_keys = [(l, j) for l in range(L) for j in range(len(wl.projections))]
     y_flat, y_views = carve([(M, wl.projections[j].N) for _, j in y_keys])
     ys = dict(zip(y_keys, y_views))
-    ws_need = max(mmf.workspace_bytes(M, p.K, p.N) for p in wl.projections)
+    by_input = {}
+    for p in wl.projections:
+        by_input.setdefault(p.input_index, []).append(p)
+    ws_need = max(max(mmf.workspace_bytes(M, ps[0].K, sum(p.N for p in ps)),  # one grouped call
+                      max(mmf.workspace_bytes(M, p.K, p.N) for p in ps))      # or single calls
+                  for ps in by_input.values())
     ws = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=dev)
     lib = mmf.lib()
 
