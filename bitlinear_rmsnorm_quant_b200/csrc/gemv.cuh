@@ -212,7 +212,15 @@ __global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_k
             if constexpr (FUSED) bulk_g2s(gamma_s, p.gamma, g_bytes, &act_bar);
             const int first = min(nst, S);
             for (int s = 0; s < first; ++s) issue_stage(s);
-            // activations may come from the previous kernel on the stream
+            // Activations may come from the previous kernel on the stream, so
+            // they are read only after it has finished; their lines are brought
+            // into L2 now (a prefetch reads nothing into this CTA, and L2 stays
+            // coherent with whatever that kernel still writes).
+            {
+                const uint8_t* xb = FUSED ? reinterpret_cast<const uint8_t*>(p.x) : reinterpret_cast<const uint8_t*>(p.q_in);
+                for (uint32_t off = 0; off < x_bytes; off += 65536u)
+                    bulk_prefetch_l2(xb + off, x_bytes - off < 65536u ? x_bytes - off : 65536u);
+            }
             pdl_wait();
             bulk_g2s(x_s, FUSED ? static_cast<const void*>(p.x) : static_cast<const void*>(p.q_in), x_bytes, &act_bar);
             pdl_launch_dependents();
