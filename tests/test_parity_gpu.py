@@ -216,6 +216,42 @@ def test_zero_and_degenerate_tokens(oracle):
     assert (y[3] == 0).all()
 
 
+@pytest.mark.parametrize("case", ["random", "zero", "constant", "tie", "near_tie", "outlier", "negative_max"])
+def test_single_token_matches_large_m_path(oracle, case):
+    """M = 1 (decode kernel, which may take the absmax from the largest |x gamma|
+    product) against the same token replicated to M = 16 (separate quantiser and
+    tensor-core kernel, full absmax reduction): the same bits, and the oracle."""
+    K, N = 2560, 512
+    x, g, W = make_layer(21, 1, K, N)
+    if case == "zero":
+        x[:] = 0.0
+    elif case == "constant":
+        x[:] = 1.5
+    elif case == "tie":
+        x[0, 5] = 9.0
+        x[0, 900] = -9.0
+        g[5] = g[900] = 1.25
+    elif case == "near_tie":
+        x[0, 5] = 9.0
+        x[0, 900] = 9.0
+        g[5] = 1.0
+        g[900] = float(np.nextafter(np.float32(1.0), np.float32(2.0)))
+    elif case == "outlier":
+        x[0, 17] = 100.0
+    elif case == "negative_max":
+        x[0, 33] = -50.0
+        g[33] = 0.5
+    packed, scale = _pack(W)
+    xd, gd = x.to(DEV), g.to(DEV)
+    y1 = mmf.bitlinear_fwd(xd, gd, packed, scale, N, EPS)
+    y16 = mmf.bitlinear_fwd(xd.expand(16, K).contiguous(), gd, packed, scale, N, EPS)
+    torch.cuda.synchronize()
+    assert mmf.workspace_bytes(1, K, N) == 0 and mmf.workspace_bytes(16, K, N) > 0  # two different paths
+    assert torch.equal(y1[0], y16[0]) and torch.equal(y16[0], y16[15])
+    y_ref, _ = oracle.bitlinear(bits_np(x), g.numpy(), EPS, W.numpy(), EPS_W)
+    assert y_rel_error(bits_np(y1), y_ref) <= Y_REL_TOL
+
+
 def test_empty_problems():
     K, N = 256, 64
     x = torch.zeros(0, K, dtype=torch.bfloat16, device=DEV)
