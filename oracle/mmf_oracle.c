@@ -197,6 +197,16 @@ void orc_rescale(const int32_t* acc, const float* absmax, float beta,
     }
 }
 
+void orc_glu_gate(const uint16_t* g, const uint16_t* u, int64_t n, uint16_t* p) {
+    for (int64_t i = 0; i < n; ++i) {
+        const float gv = orc_bf16_to_f32(g[i]);
+        const float uv = orc_bf16_to_f32(u[i]);
+        const float sig = 1.0f / (1.0f + expf(-gv));
+        const float silu = gv * sig;
+        p[i] = orc_f64_to_bf16((double)(silu * uv));
+    }
+}
+
 int orc_bitlinear(const uint16_t* x, const float* gamma, float eps,
                   const float* W, float eps_w, int64_t M, int64_t K, int64_t N,
                   uint16_t* y, float* beta_out) {

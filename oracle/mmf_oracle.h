@@ -92,6 +92,14 @@ int orc_bitlinear(const uint16_t* x, const float* gamma, float eps,
                   const float* W, float eps_w, int64_t M, int64_t K, int64_t N,
                   uint16_t* y, float* beta_out);
 
+/* The gated product of the GLU channel mixer, the input of its down
+ * projection (datacamp.com, section "Các thành phần lõi: MLGRU và GLU": one
+ * BitLinear output goes through SiLU and is multiplied element-wise by the
+ * other).  p = bf16_rn(SiLU(g) * u), SiLU(v) = v * (1 / (1 + e^-v)), each
+ * step rounded to fp32 (the precision the CUDA path takes this decision in);
+ * g, u, p bf16 [n]. */
+void orc_glu_gate(const uint16_t* g, const uint16_t* u, int64_t n, uint16_t* p);
+
 /* Number of OpenMP threads orc_ternary_acc uses (1 when built without OpenMP). */
 int orc_num_threads(void);
 

@@ -45,6 +45,8 @@ class Oracle:
         lib.orc_rescale.restype = None
         lib.orc_bitlinear.argtypes = [_P, _P, _F, _P, _F, _I64, _I64, _I64, _P, _P]
         lib.orc_bitlinear.restype = C.c_int
+        lib.orc_glu_gate.argtypes = [_P, _P, _I64, _P]
+        lib.orc_glu_gate.restype = None
         lib.orc_num_threads.argtypes = []
         lib.orc_num_threads.restype = C.c_int
         self.lib = lib
@@ -114,6 +116,14 @@ class Oracle:
         y = np.empty((M, N), dtype=np.uint16)
         self.lib.orc_rescale(_ptr(acc), _ptr(absmax), float(beta), M, N, _ptr(y))
         return y
+
+    def glu_gate(self, g_bits: np.ndarray, u_bits: np.ndarray) -> np.ndarray:
+        g_bits = np.ascontiguousarray(g_bits, dtype=np.uint16)
+        u_bits = np.ascontiguousarray(u_bits, dtype=np.uint16)
+        assert g_bits.shape == u_bits.shape
+        p = np.empty(g_bits.shape, dtype=np.uint16)
+        self.lib.orc_glu_gate(_ptr(g_bits), _ptr(u_bits), g_bits.size, _ptr(p))
+        return p
 
     def bitlinear(self, x_bits, gamma, eps, W, eps_w):
         x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)

@@ -19,6 +19,8 @@ quantisers' error bounds and hand-worked tiny cases):
   rescale            exact powers of two, torch bf16 conversion within one ulp
   whole layer        fp64 dense product of the normalised activations with the
                      ternary weights, within the activation quantiser's bound
+  GLU gated product  scipy's logistic function (fp64) within one bf16 rounding,
+                     exact zeros, SiLU(v) - SiLU(-v) = v, saturation
 """
 from __future__ import annotations
 
@@ -311,6 +313,38 @@ def check_layer_bound(orc):
     assert (np.abs(yv - ref) <= bound + np.abs(yv) * 2.0 ** -8 + 1e-12).all()
 
 
+def check_glu_gate(orc):
+    """SiLU(g) * u against an independent SiLU (scipy's logistic function, in
+    fp64) within one bf16 rounding; exact zeros; the odd-part identity
+    SiLU(v) - SiLU(-v) = v; saturation for large |g|."""
+    from scipy.special import expit
+
+    rng = np.random.default_rng(31)
+    g = _torch_bf16_bits(rng.standard_normal(4096).astype(np.float32) * 3.0)
+    u = _torch_bf16_bits(rng.standard_normal(4096).astype(np.float32))
+    p = _bf16_bits_to_f64(orc.glu_gate(g, u))
+    gv, uv = _bf16_bits_to_f64(g), _bf16_bits_to_f64(u)
+    ref = gv * expit(gv) * uv
+    # one bf16 rounding (2^-8 relative) plus the fp32 steps before it
+    assert (np.abs(p - ref) <= np.abs(ref) * (2.0 ** -8 + 2.0 ** -20) + 1e-30).all()
+    # SiLU(0) = 0 and u = 0 give exact zeros
+    z = np.zeros(4, dtype=np.uint16)
+    assert (orc.glu_gate(z, u[:4]) == 0).all() or (_bf16_bits_to_f64(orc.glu_gate(z, u[:4])) == 0).all()
+    assert (_bf16_bits_to_f64(orc.glu_gate(g[:64], np.zeros(64, dtype=np.uint16))) == 0).all()
+    # SiLU(v) - SiLU(-v) = v, with u = 1: within two bf16 roundings
+    one = _bits_of(np.ones(256, dtype=np.float32))
+    gp = _bits_of(np.linspace(-8, 8, 256).astype(np.float32).astype(np.float64).astype(np.float32)
+                  .view(np.uint32).__and__(0xFFFF0000).view(np.float32))
+    gn = _bits_of(-_bf16_bits_to_f64(gp).astype(np.float32))
+    d = _bf16_bits_to_f64(orc.glu_gate(gp, one)) - _bf16_bits_to_f64(orc.glu_gate(gn, one))
+    v = _bf16_bits_to_f64(gp)
+    assert (np.abs(d - v) <= np.abs(v) * 2.0 ** -7 + 1e-30).all()
+    # saturation: SiLU(30) = 30 to fp32 precision; SiLU(-30) is about -2.8e-12
+    big = _bits_of(np.array([30.0, -30.0], dtype=np.float32))
+    pb = _bf16_bits_to_f64(orc.glu_gate(big, _bits_of(np.array([2.0, 2.0], dtype=np.float32))))
+    assert pb[0] == 60.0 and -1e-10 < pb[1] < 0.0
+
+
 ALL_CHECKS = [
     check_bf16_rounding,
     check_absmean_worked_ties,
@@ -326,4 +360,5 @@ ALL_CHECKS = [
     check_acc_invariants,
     check_rescale,
     check_layer_bound,
+    check_glu_gate,
 ]

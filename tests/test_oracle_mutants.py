@@ -36,6 +36,8 @@ MUTANTS = [
      "for (int64_t i = 0; i < n; ++i) s += (double)W[i];"),
     ("bf16-truncate", "double s = nearbyint(ldexp(m, 8));", "double s = floor(ldexp(m, 8));"),
     ("code-offset", "const uint32_t code = (uint32_t)(t + 1);", "const uint32_t code = (uint32_t)(t & 3);"),
+    ("sigmoid-sign", "const float sig = 1.0f / (1.0f + expf(-gv));", "const float sig = 1.0f / (1.0f + expf(gv));"),
+    ("gate-on-u", "const float silu = gv * sig;", "const float silu = uv * sig;"),
 ]
 
 
