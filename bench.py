@@ -277,6 +277,22 @@ def run_ours(args, dist: Dist):
         for idx, js in sorted(groups.items()):
             K = wl.projections[js[0]].K
             x, g = xs[l, idx], gs[l, idx]
+            names = [wl.projections[j].name for j in js]
+            if args.glu and names == ["down"]:
+                # the channel mixer's down projection reads this layer set's gate and up
+                # outputs through the fused GLU call (SiLU(g) * u formed while normalising)
+                jg = [j for j, p in enumerate(wl.projections) if p.name == "gate"][0]
+                ju = [j for j, p in enumerate(wl.projections) if p.name == "up"][0]
+                j = js[0]
+                p = wl.projections[j]
+                calls.append((lib.mmf_bitlinear_fwd_glu, (ys[l, jg].data_ptr(), ys[l, ju].data_ptr(), g.data_ptr(),
+                                                          wl.eps, packed[l, j].data_ptr(), scales[l, j].data_ptr(),
+                                                          M, p.K, p.N, ys[l, j].data_ptr(), ws.data_ptr(), ws.numel(),
+                                                          flags)))
+                launches_per_step += 1 if mmf.workspace_bytes(M, p.K, p.N) == 0 else 2
+                bytes_per_step += p.N * p.K // 4 + 2 * M * p.N + 4 + 2 * (2 * M * K) + 4 * K  # g and u, gamma
+                ops_per_step += proj_ops(M, p.K, p.N)
+                continue
             if args.api == "group":
                 arr = mmf.projection_array([(packed[l, j], scales[l, j], ys[l, j], wl.projections[j].N) for j in js])
                 keep.append(arr)
@@ -416,6 +432,7 @@ def run_ours(args, dist: Dist):
             "graph": "one CUDA graph per step", "parallelism": f"dp{dist.world} (token-parallel replicas)",
             "api": "mmf_bitlinear_fwd_group" if args.api == "group" else "mmf_bitlinear_fwd",
             "pdl": not args.no_pdl and args.api == "group", "launches_per_step": launches_per_step,
+            "glu_down": bool(args.glu),
         },
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s (one token through one BitLinear layer set)",
@@ -525,6 +542,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--api", choices=("group", "single"), default="group",
                     help="group: one call per set of projections sharing x; single: one call per projection")
+    ap.add_argument("--glu", action="store_true",
+                    help="the down projection reads the gate/up outputs through mmf_bitlinear_fwd_glu")
     ap.add_argument("--no-pdl", action="store_true", help="plain stream-ordered launches")
     args = ap.parse_args(argv)
     if args.warmup < 3:

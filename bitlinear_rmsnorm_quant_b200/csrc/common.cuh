@@ -282,6 +282,27 @@ __device__ __forceinline__ int warp_sum_i32(int v) {
     return v;
 }
 
+// The GLU channel mixer's gated product of 8 bf16 pairs: p = bf16(SiLU(g) * u)
+// with SiLU(g) = g * (1 / (1 + e^-g)), each step rounded to fp32.
+__device__ __forceinline__ uint4 glu_gate8(const uint4 gv, const uint4 uv) {
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float pr[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float g = __uint_as_float(h ? (gw[i] & 0xFFFF0000u) : (gw[i] << 16));
+            const float u = __uint_as_float(h ? (uw[i] & 0xFFFF0000u) : (uw[i] << 16));
+            const float sig = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-g)));
+            pr[h] = __fmul_rn(__fmul_rn(g, sig), u);
+        }
+        const __nv_bfloat162 b = __floats2bfloat162_rn(pr[0], pr[1]);
+        out[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
 // q = clamp(rint(r * s), -127, 127) with an fp32 product rounded to nearest
 // even and ties to even in the conversion.
 __device__ __forceinline__ int quant_code(float r, float s) {

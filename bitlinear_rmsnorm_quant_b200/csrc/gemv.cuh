@@ -51,7 +51,8 @@ constexpr int kGemvSmemTwoCta = 110 * 1024;  // two CTAs per SM fit under this
 constexpr int kGemvSmemBudget = 220 * 1024;   // under the 227 KB per-CTA limit with the static part
 
 struct GemvParams {
-    const uint16_t* x;                      // bf16 [M][K]      (fused mode)
+    const uint16_t* x;                      // bf16 [M][K]      (fused mode; the gate g in GLU mode)
+    const uint16_t* u;                      // bf16 [M][K]      (GLU mode: p = bf16(SiLU(g) * u) is normalised)
     const float* gamma;                     // fp32 [K]         (fused mode)
     const int8_t* q_in;                     // int8 [M][K]      (contraction-only mode)
     const uint32_t* packed[kGemvMaxProj];   // [N_g][K/16]
@@ -141,7 +142,7 @@ __device__ __forceinline__ int gemv_proj_of(const GemvParams& p, int r) {
     return g;
 }
 
-template <int MT, bool FUSED>
+template <int MT, bool FUSED, bool GLU = false>
 __global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_kernel(const __grid_constant__ GemvParams p) {
     constexpr int NW = gemv_compute_warps(MT);
     extern __shared__ __align__(128) uint8_t smem[];
@@ -220,6 +221,11 @@ __global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_k
                 const uint8_t* xb = FUSED ? reinterpret_cast<const uint8_t*>(p.x) : reinterpret_cast<const uint8_t*>(p.q_in);
                 for (uint32_t off = 0; off < x_bytes; off += 65536u)
                     bulk_prefetch_l2(xb + off, x_bytes - off < 65536u ? x_bytes - off : 65536u);
+                if constexpr (GLU) {
+                    const uint8_t* ub = reinterpret_cast<const uint8_t*>(p.u);
+                    for (uint32_t off = 0; off < x_bytes; off += 65536u)
+                        bulk_prefetch_l2(ub + off, x_bytes - off < 65536u ? x_bytes - off : 65536u);
+                }
             }
             pdl_wait();
             bulk_g2s(x_s, FUSED ? static_cast<const void*>(p.x) : static_cast<const void*>(p.q_in), x_bytes, &act_bar);
@@ -257,7 +263,12 @@ __global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_k
         double s2 = 0.0;
         if (active && act_ok) {
             for (int c = tg; c < C8; c += 32 * WPT) {
-                const uint4 v = xr[c];
+                uint4 v = xr[c];
+                if constexpr (GLU) {
+                    // the GLU gated product replaces x (this thread alone reads chunk c later)
+                    v = glu_gate8(v, __ldg(reinterpret_cast<const uint4*>(p.u + static_cast<size_t>(m) * K) + c));
+                    const_cast<uint4*>(xr)[c] = v;
+                }
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {

@@ -60,6 +60,9 @@ template <int MT>
 cudaError_t set_gemv_attrs() {
     cudaError_t e = set_smem(gemv_kernel<MT, true>, kGemvSmemBudget);
     if (e == cudaSuccess) e = set_smem(gemv_kernel<MT, false>, kGemvSmemBudget);
+    if (e == cudaSuccess) e = set_smem(gemv_kernel<MT, true, true>, kGemvSmemBudget);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(gemv_kernel<MT, true, true>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     // All of the SM's unified memory as shared memory: a CTA of the next kernel
     // can then join a running one without the SM first draining to change the
     // split between L1 and shared memory (these kernels stage everything they
@@ -99,6 +102,7 @@ mmf_status device_state(DeviceState** out) {
         if (e == cudaSuccess) e = set_gemv_attrs<8>();
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_stream_kernel, quant_stream_smem(kMaxQuantStreamK));
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8>, 2 * kMaxK);  // one row of the largest K
+        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8, true>, 2 * kMaxK);
         if (e != cudaSuccess) return MMF_ERR_CUDA;
         if (!g_encode_tiled) {
             void* fn = nullptr;
@@ -228,12 +232,12 @@ mmf_status launch_tc(bool fused, const int8_t* q, const uint32_t* packed, const 
     }
 }
 
-template <bool FUSED>
+template <bool FUSED, bool GLU = false>
 mmf_status launch_gemv(const GemvParams& p, const GemvPlan& plan, cudaStream_t s, bool pdl) {
     const dim3 grid(static_cast<unsigned>(plan.grid));
     switch (p.M) {
 #define MMF_GEMV_CASE(MT) \
-    case MT: return launch(gemv_kernel<MT, FUSED>, grid, dim3(gemv_threads(MT)), plan.smem_bytes, s, pdl, p);
+    case MT: return launch(gemv_kernel<MT, FUSED, GLU>, grid, dim3(gemv_threads(MT)), plan.smem_bytes, s, pdl, p);
         MMF_GEMV_CASE(1)
         MMF_GEMV_CASE(2)
         MMF_GEMV_CASE(3)
@@ -248,10 +252,14 @@ mmf_status launch_gemv(const GemvParams& p, const GemvPlan& plan, cudaStream_t s
 }
 
 mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K, int8_t* q,
-                        float* absmax, int* qsum, cudaStream_t s, bool pdl, int num_sms) {
+                        float* absmax, int* qsum, cudaStream_t s, bool pdl, int num_sms,
+                        const uint16_t* u = nullptr) {
+    if (u)  // GLU: one CTA of 8 warps per row, forming SiLU(g) * u on the way
+        return launch(rmsnorm_quant_kernel<8, true>, dim3(static_cast<unsigned>(M)), dim3(256),
+                      static_cast<size_t>(K) * 2, s, pdl, x, gamma, eps, static_cast<int>(K), M, q, absmax, qsum, u);
     if (M < kQuantWarpRowMinM || K > kMaxQuantStreamK)  // one CTA of 8 warps per row
         return launch(rmsnorm_quant_kernel<8>, dim3(static_cast<unsigned>(M)), dim3(256), static_cast<size_t>(K) * 2,
-                      s, pdl, x, gamma, eps, static_cast<int>(K), M, q, absmax, qsum);
+                      s, pdl, x, gamma, eps, static_cast<int>(K), M, q, absmax, qsum, static_cast<const uint16_t*>(nullptr));
     // persistent: as many CTAs as fit on the SMs at once, never more than the rows need
     const size_t smem = quant_stream_smem(static_cast<int>(K));
     int per_sm = 0;
@@ -266,9 +274,10 @@ mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_
 }
 
 // The fused forward of `count` projections that share x.  Arguments checked.
+// u != null: GLU mode, x is the gate g and p = bf16(SiLU(g) * u) is the input.
 mmf_status fwd_impl(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K,
                     const mmf_projection* proj, int count, void* workspace, unsigned flags, cudaStream_t s,
-                    DeviceState* dev) {
+                    DeviceState* dev, const uint16_t* u = nullptr) {
     const bool pdl = (flags & MMF_FWD_PDL) != 0;
     int64_t R = 0;
     for (int i = 0; i < count; ++i) R += proj[i].N;
@@ -277,6 +286,7 @@ mmf_status fwd_impl(const uint16_t* x, const float* gamma, float eps, int64_t M,
     if (gemv_plan(static_cast<int>(M), static_cast<int>(K), R, dev->num_sms, &plan)) {
         GemvParams p{};
         p.x = x;
+        p.u = u;
         p.gamma = gamma;
         p.eps = eps;
         p.M = static_cast<int>(M);
@@ -296,10 +306,10 @@ mmf_status fwd_impl(const uint16_t* x, const float* gamma, float eps, int64_t M,
         p.rows_per_cta = plan.rows_per_cta;
         p.stage_bytes = plan.stage_bytes;
         p.stages = plan.stages;
-        return launch_gemv<true>(p, plan, s, pdl);
+        return u ? launch_gemv<true, true>(p, plan, s, pdl) : launch_gemv<true>(p, plan, s, pdl);
     }
     Workspace w = carve(workspace, M, K);
-    mmf_status st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s, pdl, dev->num_sms);
+    mmf_status st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s, pdl, dev->num_sms, u);
     if (st != MMF_OK) return st;
     for (int i = 0; i < count; ++i) {
         if (proj[i].N == 0) continue;
@@ -453,6 +463,31 @@ int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps, const ui
     pr.y = y;
     pr.N = N;
     return fwd_impl(x, gamma, eps, M, K, &pr, 1, workspace, 0u, static_cast<cudaStream_t>(stream), dev);
+}
+
+int mmf_bitlinear_fwd_glu(const uint16_t* g, const uint16_t* u, const float* gamma, float eps,
+                          const uint32_t* packed, const float* scale, int64_t M, int64_t K, int64_t N, uint16_t* y,
+                          void* workspace, size_t workspace_bytes, unsigned flags, void* stream) {
+    if (!(eps >= 0.0f) || eps > 1e30f) return MMF_ERR_INVALID_ARG;
+    if (flags & ~MMF_FWD_PDL) return MMF_ERR_INVALID_ARG;
+    mmf_status st = check_shape(M, K, N);
+    if (st != MMF_OK) return st;
+    if (M == 0 || N == 0) return MMF_OK;
+    if (!g || !u || !gamma || !packed || !scale || !y) return MMF_ERR_INVALID_ARG;
+    if (!aligned16(g) || !aligned16(u) || !aligned16(gamma) || !aligned16(packed) || !aligned16(scale) ||
+        !aligned16(y))
+        return MMF_ERR_MISALIGNED;
+    const size_t need = mmf_workspace_bytes(M, K, N);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return MMF_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return MMF_ERR_MISALIGNED;
+    DeviceState* dev;
+    if ((st = device_state(&dev)) != MMF_OK) return st;
+    mmf_projection pr;
+    pr.packed = packed;
+    pr.scale = scale;
+    pr.y = y;
+    pr.N = N;
+    return fwd_impl(g, gamma, eps, M, K, &pr, 1, workspace, flags, static_cast<cudaStream_t>(stream), dev, u);
 }
 
 int mmf_bitlinear_fwd_group(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K,

@@ -78,13 +78,16 @@ __host__ __device__ inline int quant_rows_per_cta(int K) {
     return r;
 }
 
-template <int WPR>
+// GLU: x is the gate g of the GLU channel mixer and the row normalised is
+// p = bf16(SiLU(g) * u), formed in pass 1 and kept in place of x.
+template <int WPR, bool GLU = false>
 __global__ void __launch_bounds__(kQuantRowsPerCta * 32) rmsnorm_quant_kernel(const uint16_t* __restrict__ x,
                                                                               const float* __restrict__ gamma,
                                                                               float eps, int K, int64_t M,
                                                                               int8_t* __restrict__ q,
                                                                               float* __restrict__ absmax,
-                                                                              int* __restrict__ qsum) {
+                                                                              int* __restrict__ qsum,
+                                                                              const uint16_t* __restrict__ u) {
     extern __shared__ __align__(128) uint4 xs_all[];  // one slice of K/8 chunks per row
     __shared__ __align__(8) uint64_t row_bar[kQuantRowsPerCta];
     __shared__ double red_d[WPR];
@@ -133,7 +136,14 @@ __global__ void __launch_bounds__(kQuantRowsPerCta * 32) rmsnorm_quant_kernel(co
     double s2[4] = {0.0, 0.0, 0.0, 0.0};
     for (int c = c0; c < C; c += cstep) {
         float f[8];
-        unpack_bf16x8(xs[c], f);
+        if constexpr (GLU) {
+            // this thread alone reads chunk c in the passes below
+            const uint4 pv = glu_gate8(xs[c], __ldg(reinterpret_cast<const uint4*>(u + m * static_cast<int64_t>(K)) + c));
+            xs[c] = pv;
+            unpack_bf16x8(pv, f);
+        } else {
+            unpack_bf16x8(xs[c], f);
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) s2[i & 3] += static_cast<double>(f[i]) * static_cast<double>(f[i]);
     }

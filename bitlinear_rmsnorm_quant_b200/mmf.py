@@ -40,6 +40,7 @@ SIGNATURES = {
     "mmf_quantize_act": (_INT, [_P, _P, _F, _I64, _I64, _P, _P, _P]),
     "mmf_ternary_acc": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "mmf_bitlinear_fwd": (_INT, [_P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "mmf_bitlinear_fwd_glu": (_INT, [_P, _P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, C.c_uint, _P]),
     "mmf_bitlinear_fwd_group": (_INT, [_P, _P, _F, _I64, _I64, _P, _INT, _P, _SZ, C.c_uint, _P]),
     "mmf_bitlinear_fwd_noalloc": (_INT, [_P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P]),
     "mmf_hbm_copy": (_INT, [_P, _P, _SZ, _P]),
@@ -187,6 +188,23 @@ def projection_array(items):
     for i, (packed, scale, y, N) in enumerate(items):
         arr[i] = Projection(packed.data_ptr(), scale.data_ptr(), y.data_ptr() if y is not None else None, N)
     return arr
+
+
+def bitlinear_fwd_glu(g: torch.Tensor, u: torch.Tensor, gamma: torch.Tensor, packed: torch.Tensor,
+                      scale: torch.Tensor, N: int, eps: float = 1e-6, workspace=None, out=None, flags: int = 0,
+                      stream=None):
+    """GLU down projection: bf16 g[M, K], u[M, K] -> bf16 y[M, N] of BitLinear(bf16(SiLU(g) * u))."""
+    _dev(g, torch.bfloat16, "g")
+    _dev(u, torch.bfloat16, "u")
+    M, K = g.shape
+    assert u.shape == g.shape
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=g.device)
+    ws, ws_n = _workspace(M, K, N, g.device, workspace)
+    check(lib().mmf_bitlinear_fwd_glu(g.data_ptr(), u.data_ptr(), gamma.data_ptr(), eps, packed.data_ptr(),
+                                      scale.data_ptr(), M, K, N, y.data_ptr(),
+                                      ws.data_ptr() if ws is not None else None, ws_n, flags, _stream(stream)),
+          "mmf_bitlinear_fwd_glu")
+    return y
 
 
 def bitlinear_fwd_group(x: torch.Tensor, gamma: torch.Tensor, weights, eps: float = 1e-6, workspace=None,

@@ -141,6 +141,26 @@ int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps,
                       int64_t K, int64_t N, uint16_t* y, void* workspace,
                       size_t workspace_bytes, void* stream);
 
+/*
+ * mmf_bitlinear_fwd_glu -- the down projection of the GLU channel mixer with
+ * its gating fused in (datacamp.com, section "Các thành phần lõi: MLGRU và
+ * GLU": the input goes through two BitLinear layers, one output through
+ * SiLU, multiplied element-wise by the other, and the product through a
+ * third BitLinear layer).  The input of the fused forward is
+ *   p[m][k] = bf16_rn(SiLU(g[m][k]) * u[m][k]),  SiLU(v) = v * (1 / (1 + e^-v)),
+ * each step rounded to fp32; then as mmf_bitlinear_fwd with x = p.  p never
+ * goes to memory: the kernels form it while normalising.
+ * g, u: bf16 [M][K] (the gate and up projections' outputs); other arguments,
+ * workspace (mmf_workspace_bytes(M, K, N)) and errors as mmf_bitlinear_fwd;
+ * flags: 0 or MMF_FWD_PDL (g and u are then read only after the kernel before
+ * has finished, like x).  g, u, y and the workspace must not overlap.
+ */
+int mmf_bitlinear_fwd_glu(const uint16_t* g, const uint16_t* u,
+                          const float* gamma, float eps, const uint32_t* packed,
+                          const float* scale, int64_t M, int64_t K, int64_t N,
+                          uint16_t* y, void* workspace, size_t workspace_bytes,
+                          unsigned flags, void* stream);
+
 /* Flags of mmf_bitlinear_fwd_group. */
 #define MMF_FWD_PDL 1u   /* launch as a programmatic dependent of the kernel before it on the stream (see below) */
 #define MMF_MAX_GROUP 8  /* projections per mmf_bitlinear_fwd_group call */

@@ -133,3 +133,14 @@ def test_group_argument_errors(L):
     assert f(None, None, 1e-6, 1, 128, arr, 1, None, 0, 0, None) == 0     # empty group
     arr[0] = mmf.Projection(A, A, A, 16)
     assert f(A, A, 1e-6, 4096, 2048, arr, 1, None, 0, 0, None) == 4       # large M needs workspace
+
+
+def test_glu_argument_errors(L):
+    f = L.mmf_bitlinear_fwd_glu
+    assert f(A, None, A, 1e-6, A, A, 1, 128, 16, A, None, 0, 0, None) == 1      # no u
+    assert f(A, A, A, 1e-6, A, A, 1, 128, 16, A, None, 0, 2, None) == 1        # unknown flag
+    assert f(A, A, A, -1.0, A, A, 1, 128, 16, A, None, 0, 0, None) == 1        # bad eps
+    assert f(A, A, A, 1e-6, A, A, 1, 100, 16, A, None, 0, 0, None) == 2        # bad K
+    assert f(A, MIS, A, 1e-6, A, A, 1, 128, 16, A, None, 0, 0, None) == 3      # misaligned u
+    assert f(A, A, A, 1e-6, A, A, 4096, 2048, 2048, A, None, 0, 0, None) == 4  # missing workspace
+    assert f(None, None, None, 1e-6, None, None, 0, 128, 16, None, None, 0, 0, None) == 0  # empty

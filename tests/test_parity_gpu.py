@@ -252,6 +252,48 @@ def test_single_token_matches_large_m_path(oracle, case):
     assert y_rel_error(bits_np(y1), y_ref) <= Y_REL_TOL
 
 
+# -- GLU channel mixer: down projection with SiLU(g) * u fused in -----------------------------
+
+@pytest.mark.parametrize("M,K,N", [(1, 6912, 2560), (3, 2816, 1024), (8, 5632, 2048), (1, 128, 16),
+                                   (64, 2816, 1024), (300, 6912, 640), (4100, 1024, 256)])
+def test_glu_parity(oracle, M, K, N):
+    """y of the fused GLU call against the oracle's gated product fed to its BitLinear."""
+    g, gamma, W = make_layer(22, M, K, N)
+    u = I.activations(22, M, K, index=5)
+    packed, scale = _pack(W)
+    y = mmf.bitlinear_fwd_glu(g.to(DEV), u.to(DEV), gamma.to(DEV), packed, scale, N, EPS)
+    torch.cuda.synchronize()
+    p_bits = oracle.glu_gate(bits_np(g), bits_np(u))
+    y_ref, beta = oracle.bitlinear(p_bits, gamma.numpy(), EPS, W.numpy(), EPS_W)
+    assert np.float32(scale.item()) == beta
+    assert y_rel_error(bits_np(y), y_ref) <= Y_REL_TOL
+
+
+def test_glu_paths_agree_and_match_plain_call():
+    """One token on the decode kernel, the same token replicated on the large-M
+    path, with and without PDL: identical bits.  And the fused call equals the
+    plain call given the gated product the GPU forms (read back through the
+    large-M path's own rounding: the same fp32 steps)."""
+    K, N = 2816, 512
+    g, gamma, W = make_layer(23, 1, K, N)
+    u = I.activations(23, 1, K, index=6)
+    packed, scale = _pack(W)
+    gd, ud, gmd = g.to(DEV), u.to(DEV), gamma.to(DEV)
+    y1 = mmf.bitlinear_fwd_glu(gd, ud, gmd, packed, scale, N, EPS)
+    y1p = mmf.bitlinear_fwd_glu(gd, ud, gmd, packed, scale, N, EPS, flags=mmf.FWD_PDL)
+    y16 = mmf.bitlinear_fwd_glu(gd.expand(16, K).contiguous(), ud.expand(16, K).contiguous(), gmd, packed, scale, N,
+                                EPS)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y1p) and torch.equal(y1[0], y16[0]) and torch.equal(y16[0], y16[15])
+    # the plain call on p computed on the host in the same fp32 steps agrees within the tolerance
+    gf, uf = g.float(), u.float()
+    p = (gf * (1.0 / (1.0 + torch.exp(-gf))) * uf).to(torch.bfloat16)
+    y_plain = mmf.bitlinear_fwd(p.to(DEV), gmd, packed, scale, N, EPS)
+    torch.cuda.synchronize()
+    yv, yp = y1.float().cpu().numpy(), y_plain.float().cpu().numpy()
+    assert np.abs(yv - yp).max() <= 1e-2 * max(np.abs(yp).max(), 1e-6)
+
+
 def test_empty_problems():
     K, N = 256, 64
     x = torch.zeros(0, K, dtype=torch.bfloat16, device=DEV)
