@@ -3,8 +3,9 @@
 // item "RMS norm"; fused so x is read from HBM once: ld246.com, section
 // "融合 BitLinear 层的创新").
 //
-// One warp per token row.  The row is copied from HBM once into shared
-// memory, then:
+// Each token row is copied from HBM once into shared memory (a persistent
+// streaming kernel with one warp per row for large M; one 8-warp CTA per row
+// otherwise), then:
 //   ms  = (float)(sum x^2 / K)         fp64 sum (bf16 squares are exact in fp64)
 //   inv = 1 / sqrt(ms + eps)           fp32, correctly rounded
 //   r   = (x * inv) * gamma            fp32, two roundings
@@ -58,30 +59,21 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& v, float (&f)[8]) {
     }
 }
 
-// WPR warps per token row; a CTA holds kQuantRowsPerCta rows when WPR == 1,
-// else one row.  One thread brings the whole row into shared memory with bulk
+// WPR warps per token row, one row per CTA when WPR > 1 (the library launches
+// WPR = 8: below 4096 rows, for K above the streaming kernel's limit, and in
+// GLU mode).  One thread brings the whole row into shared memory with bulk
 // copies (one request per row, so the row's HBM latency is paid once, not once
-// per 16-byte load); the three passes then run from shared memory.  With one
-// warp per row there is no CTA-wide barrier, so the rows of a CTA proceed
-// independently and the staged bytes per CTA are capped so that at least two
-// CTAs fit on an SM at any K; that form is for large M.  Small M takes 8 warps
-// per row to spread the arithmetic over more SMs.
-constexpr int kQuantRowsPerCta = 8;
-constexpr int kQuantSmemBudget = 112 * 1024;
+// per 16-byte load); the three passes then run from shared memory, reduced
+// across the row's warps in index order.  With WPR = 1 a CTA holds one row per
+// warp and needs no CTA-wide barrier.
+constexpr int kQuantCtaWarps = 8;
 constexpr uint32_t kQuantPieceBytes = 32 * 1024;  // bytes per bulk copy request
-constexpr int64_t kQuantWarpRowMinM = 4096;       // rows from which one warp per row pays
-
-__host__ __device__ inline int quant_rows_per_cta(int K) {
-    int r = kQuantSmemBudget / (2 * K);
-    if (r > kQuantRowsPerCta) r = kQuantRowsPerCta;
-    if (r < 1) r = 1;
-    return r;
-}
+constexpr int64_t kQuantWarpRowMinM = 4096;       // rows from which the streaming kernel takes over
 
 // GLU: x is the gate g of the GLU channel mixer and the row normalised is
 // p = bf16(SiLU(g) * u), formed in pass 1 and kept in place of x.
 template <int WPR, bool GLU = false>
-__global__ void __launch_bounds__(kQuantRowsPerCta * 32) rmsnorm_quant_kernel(const uint16_t* __restrict__ x,
+__global__ void __launch_bounds__(kQuantCtaWarps * 32) rmsnorm_quant_kernel(const uint16_t* __restrict__ x,
                                                                               const float* __restrict__ gamma,
                                                                               float eps, int K, int64_t M,
                                                                               int8_t* __restrict__ q,
@@ -89,7 +81,7 @@ __global__ void __launch_bounds__(kQuantRowsPerCta * 32) rmsnorm_quant_kernel(co
                                                                               int* __restrict__ qsum,
                                                                               const uint16_t* __restrict__ u) {
     extern __shared__ __align__(128) uint4 xs_all[];  // one slice of K/8 chunks per row
-    __shared__ __align__(8) uint64_t row_bar[kQuantRowsPerCta];
+    __shared__ __align__(8) uint64_t row_bar[kQuantCtaWarps];
     __shared__ double red_d[WPR];
     __shared__ float red_f[WPR];
     __shared__ int red_i[WPR];
