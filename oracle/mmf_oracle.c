@@ -207,6 +207,27 @@ void orc_glu_gate(const uint16_t* g, const uint16_t* u, int64_t n, uint16_t* p) 
     }
 }
 
+static float orc_sigmoid(float v) { return 1.0f / (1.0f + expf(-v)); }
+
+void orc_mlgru_scan(const uint16_t* f_pre, const uint16_t* c_pre, const uint16_t* g_pre,
+                    const float* h0, int64_t B, int64_t T, int64_t D, uint16_t* o, float* h_last) {
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t k = 0; k < D; ++k) {
+            float h = h0 ? h0[b * D + k] : 0.0f;
+            for (int64_t t = 0; t < T; ++t) {
+                const int64_t i = (b * T + t) * D + k;
+                const float f = orc_sigmoid(orc_bf16_to_f32(f_pre[i]));
+                const float cv = orc_bf16_to_f32(c_pre[i]);
+                const float c = cv * orc_sigmoid(cv);
+                const float g = orc_sigmoid(orc_bf16_to_f32(g_pre[i]));
+                h = f * h + (1.0f - f) * c;
+                o[i] = orc_f64_to_bf16((double)(g * h));
+            }
+            h_last[b * D + k] = h;
+        }
+    }
+}
+
 int orc_bitlinear(const uint16_t* x, const float* gamma, float eps,
                   const float* W, float eps_w, int64_t M, int64_t K, int64_t N,
                   uint16_t* y, float* beta_out) {

@@ -100,6 +100,19 @@ int orc_bitlinear(const uint16_t* x, const float* gamma, float eps,
  * g, u, p bf16 [n]. */
 void orc_glu_gate(const uint16_t* g, const uint16_t* u, int64_t n, uint16_t* p);
 
+/* The MLGRU token mixer's element-wise recurrence (datacamp.com, section
+ * "Các thành phần lõi: MLGRU và GLU": tokens are taken one at a time; gates
+ * with values between 0 and 1 decide how much of the previous hidden state and
+ * of the current token is kept; jiqizhixin.com, section "MatMul-free 语言模型
+ * 架构", whose formulas are stripped).  For every sequence b and channel k,
+ * from h = h0[b][k] (0 when h0 is NULL), token by token:
+ *   f = sigma(f_pre), c = SiLU(c_pre), g = sigma(g_pre),  sigma(v) = 1 / (1 + e^-v),
+ *   h = f * h + (1 - f) * c,  o = bf16_rn(g * h)
+ * every step rounded to fp32; h_last[b][k] = h after the last token.
+ * f_pre, c_pre, g_pre, o: bf16 [B][T][D]; h0, h_last: fp32 [B][D]. */
+void orc_mlgru_scan(const uint16_t* f_pre, const uint16_t* c_pre, const uint16_t* g_pre,
+                    const float* h0, int64_t B, int64_t T, int64_t D, uint16_t* o, float* h_last);
+
 /* Number of OpenMP threads orc_ternary_acc uses (1 when built without OpenMP). */
 int orc_num_threads(void);
 

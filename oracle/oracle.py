@@ -47,6 +47,8 @@ class Oracle:
         lib.orc_bitlinear.restype = C.c_int
         lib.orc_glu_gate.argtypes = [_P, _P, _I64, _P]
         lib.orc_glu_gate.restype = None
+        lib.orc_mlgru_scan.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]
+        lib.orc_mlgru_scan.restype = None
         lib.orc_num_threads.argtypes = []
         lib.orc_num_threads.restype = C.c_int
         self.lib = lib
@@ -124,6 +126,21 @@ class Oracle:
         p = np.empty(g_bits.shape, dtype=np.uint16)
         self.lib.orc_glu_gate(_ptr(g_bits), _ptr(u_bits), g_bits.size, _ptr(p))
         return p
+
+    def mlgru_scan(self, f_bits, c_bits, g_bits, h0=None):
+        """bf16 [B, T, D] pre-activations -> (o bf16 bits [B, T, D], h_last fp32 [B, D])."""
+        f_bits = np.ascontiguousarray(f_bits, dtype=np.uint16)
+        c_bits = np.ascontiguousarray(c_bits, dtype=np.uint16)
+        g_bits = np.ascontiguousarray(g_bits, dtype=np.uint16)
+        B, T, D = f_bits.shape
+        o = np.empty((B, T, D), dtype=np.uint16)
+        h_last = np.empty((B, D), dtype=np.float32)
+        h0p = None
+        if h0 is not None:
+            h0 = np.ascontiguousarray(h0, dtype=np.float32)
+            h0p = _ptr(h0)
+        self.lib.orc_mlgru_scan(_ptr(f_bits), _ptr(c_bits), _ptr(g_bits), h0p, B, T, D, _ptr(o), _ptr(h_last))
+        return o, h_last
 
     def bitlinear(self, x_bits, gamma, eps, W, eps_w):
         x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)

@@ -21,6 +21,8 @@ quantisers' error bounds and hand-worked tiny cases):
                      ternary weights, within the activation quantiser's bound
   GLU gated product  scipy's logistic function (fp64) within one bf16 rounding,
                      exact zeros, SiLU(v) - SiLU(-v) = v, saturation
+  MLGRU recurrence   closed form for constant gates and inputs, forgetting and
+                     keeping limits, continuation across calls, independence
 """
 from __future__ import annotations
 
@@ -345,6 +347,45 @@ def check_glu_gate(orc):
     assert pb[0] == 60.0 and -1e-10 < pb[1] < 0.0
 
 
+def check_mlgru_scan(orc):
+    """The recurrence against closed forms: constant gates and inputs give
+    h_t = c + f^t (h0 - c); f -> 0 forgets (h_t = SiLU(c_t)); f -> 1 keeps h0;
+    the output gate at 0 pre-activation halves h; sequences and channels are
+    independent; h_last continues the recurrence across calls."""
+    B, T, D = 2, 40, 3
+
+    def bits(v):
+        return _bits_of(np.full((B, T, D), v, dtype=np.float32))
+
+    sig = lambda v: 1.0 / (1.0 + math.exp(-v))
+    # constant f_pre = 0.5, c_pre = 2.0, g_pre = 0: closed form
+    h0 = np.array([[1.5, -2.0, 0.0], [4.0, 0.25, -1.0]], dtype=np.float32)
+    o, hl = orc.mlgru_scan(bits(0.5), bits(2.0), bits(0.0), h0)
+    f, c = sig(0.5), 2.0 * sig(2.0)
+    for t in range(T):
+        ref = c + f ** (t + 1) * (h0.astype(np.float64) - c)
+        assert np.allclose(_bf16_bits_to_f64(o[:, t, :]), 0.5 * ref, rtol=2.0 ** -7, atol=1e-6)
+    assert np.allclose(hl, c + f ** T * (h0.astype(np.float64) - c), rtol=1e-5, atol=1e-6)
+    # f -> 0 (f_pre = -64): no memory, h_t = SiLU(c_t); f -> 1 (f_pre = 64): h stays h0
+    rng = np.random.default_rng(41)
+    cb = _torch_bf16_bits(rng.standard_normal((B, T, D)).astype(np.float32))
+    o, hl = orc.mlgru_scan(bits(-64.0), cb, bits(64.0), h0)
+    cv = _bf16_bits_to_f64(cb)
+    assert np.allclose(_bf16_bits_to_f64(o), cv / (1.0 + np.exp(-cv)), rtol=2.0 ** -7, atol=1e-30)
+    o, hl = orc.mlgru_scan(bits(64.0), cb, bits(64.0), h0)
+    assert np.allclose(_bf16_bits_to_f64(o), np.broadcast_to(h0[:, None, :], (B, T, D)), rtol=2.0 ** -7)
+    assert np.array_equal(hl, h0)
+    # independence and continuation: two halves with h_last carried equal one call
+    fb = _torch_bf16_bits(rng.standard_normal((B, T, D)).astype(np.float32))
+    gb = _torch_bf16_bits(rng.standard_normal((B, T, D)).astype(np.float32))
+    o_all, h_all = orc.mlgru_scan(fb, cb, gb, h0)
+    o1, h1 = orc.mlgru_scan(fb[:, :17], cb[:, :17], gb[:, :17], h0)
+    o2, h2 = orc.mlgru_scan(fb[:, 17:], cb[:, 17:], gb[:, 17:], h1)
+    assert np.array_equal(o_all, np.concatenate([o1, o2], axis=1)) and np.array_equal(h_all, h2)
+    o_b1, _ = orc.mlgru_scan(fb[1:], cb[1:], gb[1:], h0[1:])
+    assert np.array_equal(o_all[1:], o_b1)
+
+
 ALL_CHECKS = [
     check_bf16_rounding,
     check_absmean_worked_ties,
@@ -361,4 +402,5 @@ ALL_CHECKS = [
     check_rescale,
     check_layer_bound,
     check_glu_gate,
+    check_mlgru_scan,
 ]

@@ -38,6 +38,9 @@ MUTANTS = [
     ("code-offset", "const uint32_t code = (uint32_t)(t + 1);", "const uint32_t code = (uint32_t)(t & 3);"),
     ("sigmoid-sign", "const float sig = 1.0f / (1.0f + expf(-gv));", "const float sig = 1.0f / (1.0f + expf(gv));"),
     ("gate-on-u", "const float silu = gv * sig;", "const float silu = uv * sig;"),
+    ("forget-swapped", "h = f * h + (1.0f - f) * c;", "h = (1.0f - f) * h + f * c;"),
+    ("no-output-gate", "o[i] = orc_f64_to_bf16((double)(g * h));", "o[i] = orc_f64_to_bf16((double)h);"),
+    ("silu-as-sigmoid", "const float c = cv * orc_sigmoid(cv);", "const float c = orc_sigmoid(cv);"),
 ]
 
 
