@@ -14,6 +14,7 @@
 #include "gemv.cuh"
 #include "pack.cuh"
 #include "quant.cuh"
+#include "scan.cuh"
 
 namespace {
 
@@ -463,6 +464,25 @@ int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps, const ui
     pr.y = y;
     pr.N = N;
     return fwd_impl(x, gamma, eps, M, K, &pr, 1, workspace, 0u, static_cast<cudaStream_t>(stream), dev);
+}
+
+int mmf_mlgru_scan(const uint16_t* f_pre, const uint16_t* c_pre, const uint16_t* g_pre, const float* h0, int64_t B,
+                   int64_t T, int64_t D, uint16_t* o, float* h_last, void* stream) {
+    if (B < 0 || T < 0 || D < 0) return MMF_ERR_INVALID_ARG;
+    if ((D % 2) != 0 || D > kMaxDim || T > kMaxDim || B > 65535 || B * T * D > (int64_t(1) << 40))
+        return MMF_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0 || D == 0) return MMF_OK;
+    if (T > 0 && (!f_pre || !c_pre || !g_pre || !o)) return MMF_ERR_INVALID_ARG;
+    if (T == 0 && !h_last) return MMF_OK;
+    if (!aligned16(f_pre) || !aligned16(c_pre) || !aligned16(g_pre) || !aligned16(o) || !aligned16(h0) ||
+        !aligned16(h_last))
+        return MMF_ERR_MISALIGNED;
+    DeviceState* dev;
+    mmf_status st = device_state(&dev);
+    if (st != MMF_OK) return st;
+    const dim3 grid(static_cast<unsigned>((D + 63) / 64), static_cast<unsigned>(B));
+    return launch(mlgru_scan_kernel, grid, dim3(kScanWarps * 32), 0, static_cast<cudaStream_t>(stream), false, f_pre,
+                  c_pre, g_pre, h0, static_cast<int>(T), static_cast<int>(D), o, h_last);
 }
 
 int mmf_bitlinear_fwd_glu(const uint16_t* g, const uint16_t* u, const float* gamma, float eps,

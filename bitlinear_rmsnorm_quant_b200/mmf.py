@@ -41,6 +41,7 @@ SIGNATURES = {
     "mmf_ternary_acc": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "mmf_bitlinear_fwd": (_INT, [_P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "mmf_bitlinear_fwd_glu": (_INT, [_P, _P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, C.c_uint, _P]),
+    "mmf_mlgru_scan": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P]),
     "mmf_bitlinear_fwd_group": (_INT, [_P, _P, _F, _I64, _I64, _P, _INT, _P, _SZ, C.c_uint, _P]),
     "mmf_bitlinear_fwd_noalloc": (_INT, [_P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P]),
     "mmf_hbm_copy": (_INT, [_P, _P, _SZ, _P]),
@@ -205,6 +206,20 @@ def bitlinear_fwd_glu(g: torch.Tensor, u: torch.Tensor, gamma: torch.Tensor, pac
                                       ws.data_ptr() if ws is not None else None, ws_n, flags, _stream(stream)),
           "mmf_bitlinear_fwd_glu")
     return y
+
+
+def mlgru_scan(f_pre: torch.Tensor, c_pre: torch.Tensor, g_pre: torch.Tensor, h0: torch.Tensor | None = None,
+               out=None, h_last=None, stream=None):
+    """MLGRU recurrence: bf16 [B, T, D] pre-activations -> (bf16 o [B, T, D], fp32 h_last [B, D])."""
+    for name, t in (("f_pre", f_pre), ("c_pre", c_pre), ("g_pre", g_pre)):
+        _dev(t, torch.bfloat16, name)
+    B, T, D = f_pre.shape
+    o = out if out is not None else torch.empty((B, T, D), dtype=torch.bfloat16, device=f_pre.device)
+    hl = h_last if h_last is not None else torch.empty((B, D), dtype=torch.float32, device=f_pre.device)
+    check(lib().mmf_mlgru_scan(f_pre.data_ptr(), c_pre.data_ptr(), g_pre.data_ptr(),
+                               h0.data_ptr() if h0 is not None else None, B, T, D, o.data_ptr(), hl.data_ptr(),
+                               _stream(stream)), "mmf_mlgru_scan")
+    return o, hl
 
 
 def bitlinear_fwd_group(x: torch.Tensor, gamma: torch.Tensor, weights, eps: float = 1e-6, workspace=None,

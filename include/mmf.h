@@ -161,6 +161,28 @@ int mmf_bitlinear_fwd_glu(const uint16_t* g, const uint16_t* u,
                           uint16_t* y, void* workspace, size_t workspace_bytes,
                           unsigned flags, void* stream);
 
+/*
+ * mmf_mlgru_scan -- the MLGRU token mixer's element-wise recurrence between
+ * its f/c/g projections and its o projection (datacamp.com, section "Các
+ * thành phần lõi: MLGRU và GLU": tokens taken one at a time, gates in (0, 1)
+ * deciding how much of the previous hidden state and of the current token is
+ * kept).  For every sequence b and channel k, from h = h0[b][k] (0 when h0 is
+ * NULL), token by token:
+ *   f = sigma(f_pre), c = SiLU(c_pre), g = sigma(g_pre),  sigma(v) = 1/(1 + e^-v)
+ *   h = f * h + (1 - f) * c          (fp32)
+ *   o[b][t][k] = bf16_rn(g * h)      (the o projection's input)
+ * and h_last[b][k] = h after the last token (may be NULL).  Tokens are split
+ * into chunks combined through their linear maps h -> A h + B, so the result
+ * matches the token-by-token recurrence to fp32 rounding, not bit for bit.
+ * f_pre, c_pre, g_pre, o: bf16 [B][T][D] (the projections' y layout with
+ * M = B * T); h0, h_last: fp32 [B][D].  D must be even, B <= 65535; pointers
+ * 16-byte aligned; o must not overlap the inputs.  T = 0 copies h0 (or zeros)
+ * to h_last.
+ */
+int mmf_mlgru_scan(const uint16_t* f_pre, const uint16_t* c_pre,
+                   const uint16_t* g_pre, const float* h0, int64_t B, int64_t T,
+                   int64_t D, uint16_t* o, float* h_last, void* stream);
+
 /* Flags of mmf_bitlinear_fwd_group. */
 #define MMF_FWD_PDL 1u   /* launch as a programmatic dependent of the kernel before it on the stream (see below) */
 #define MMF_MAX_GROUP 8  /* projections per mmf_bitlinear_fwd_group call */

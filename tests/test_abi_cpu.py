@@ -144,3 +144,12 @@ def test_glu_argument_errors(L):
     assert f(A, MIS, A, 1e-6, A, A, 1, 128, 16, A, None, 0, 0, None) == 3      # misaligned u
     assert f(A, A, A, 1e-6, A, A, 4096, 2048, 2048, A, None, 0, 0, None) == 4  # missing workspace
     assert f(None, None, None, 1e-6, None, None, 0, 128, 16, None, None, 0, 0, None) == 0  # empty
+
+
+def test_mlgru_scan_argument_errors(L):
+    f = L.mmf_mlgru_scan
+    assert f(A, A, A, None, 1, 4, 65, A, A, None) == 2      # odd D
+    assert f(A, A, A, None, -1, 4, 64, A, A, None) == 1     # negative size
+    assert f(A, None, A, None, 1, 4, 64, A, A, None) == 1   # missing input
+    assert f(A, A, A, MIS, 1, 4, 64, A, A, None) == 3       # misaligned h0
+    assert f(None, None, None, None, 0, 4, 64, None, None, None) == 0  # empty

@@ -13,7 +13,8 @@ import torch
 from bitlinear_rmsnorm_quant_b200 import mmf
 from bitlinear_rmsnorm_quant_b200 import inputs as I
 from bitlinear_rmsnorm_quant_b200 import workloads as WL
-from gpu_cases import (Q_MAX_DIFF_FRAC, Y_REL_TOL, bits_np, make_layer, q_diff_stats, y_rel_error)
+from gpu_cases import (Q_MAX_DIFF_FRAC, Y_REL_TOL, bf16_to_f64, bits_np, make_layer, q_diff_stats,
+                       y_rel_error)
 
 pytestmark = pytest.mark.gpu
 
@@ -292,6 +293,45 @@ def test_glu_paths_agree_and_match_plain_call():
     torch.cuda.synchronize()
     yv, yp = y1.float().cpu().numpy(), y_plain.float().cpu().numpy()
     assert np.abs(yv - yp).max() <= 1e-2 * max(np.abs(yp).max(), 1e-6)
+
+
+# -- MLGRU token mixer recurrence -------------------------------------------------------------
+
+@pytest.mark.parametrize("B,T,D", [(1, 1, 2560), (2, 37, 128), (3, 100, 66), (4, 2048, 2048), (2, 5, 64),
+                                   (1, 0, 64)])
+@pytest.mark.parametrize("with_h0", [False, True])
+def test_mlgru_scan_parity(oracle, B, T, D, with_h0):
+    rng = np.random.default_rng(B * 1000 + T + D)
+    mk = lambda: torch.from_numpy(rng.standard_normal((B, T, D)).astype(np.float32) * 2.0).to(torch.bfloat16)
+    fp, cp, gp = mk(), mk(), mk()
+    h0 = torch.from_numpy(rng.standard_normal((B, D)).astype(np.float32)) if with_h0 else None
+    o, hl = mmf.mlgru_scan(fp.to(DEV), cp.to(DEV), gp.to(DEV), h0.to(DEV) if with_h0 else None)
+    torch.cuda.synchronize()
+    o_ref, hl_ref = oracle.mlgru_scan(bits_np(fp), bits_np(cp), bits_np(gp), h0.numpy() if with_h0 else None)
+    ov, rv = bf16_to_f64(bits_np(o.cpu())), bf16_to_f64(o_ref)
+    # chunked combination rounds differently from token-by-token: within fp32
+    # rounding of the state, then at most one bf16 step of o
+    h_tol = 1e-4 * (1.0 + np.abs(hl_ref))
+    assert (np.abs(hl.cpu().numpy() - hl_ref) <= h_tol).all()
+    assert (np.abs(ov - rv) <= np.abs(rv) * 2.0 ** -7 + 1e-6).all()
+    if T > 0:
+        assert (ov == rv).mean() > 0.99
+
+
+def test_mlgru_scan_continues_across_calls():
+    """Two calls over the halves of the tokens, the state carried, give the
+    single call's output to fp32 rounding of the state."""
+    B, T, D = 2, 300, 256
+    rng = np.random.default_rng(7)
+    mk = lambda: torch.from_numpy(rng.standard_normal((B, T, D)).astype(np.float32)).to(torch.bfloat16).to(DEV)
+    fp, cp, gp = mk(), mk(), mk()
+    o, hl = mmf.mlgru_scan(fp, cp, gp)
+    o1, h1 = mmf.mlgru_scan(fp[:, :120].contiguous(), cp[:, :120].contiguous(), gp[:, :120].contiguous())
+    o2, h2 = mmf.mlgru_scan(fp[:, 120:].contiguous(), cp[:, 120:].contiguous(), gp[:, 120:].contiguous(), h1)
+    torch.cuda.synchronize()
+    assert torch.allclose(hl, h2, rtol=1e-4, atol=1e-4)
+    both = torch.cat([o1, o2], dim=1).float()
+    assert ((both - o.float()).abs() <= o.float().abs() * 2.0 ** -7 + 1e-6).all()
 
 
 def test_empty_problems():
