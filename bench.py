@@ -67,6 +67,102 @@ def load_peaks():
                 "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def run_scan(args, dist):
+    """The MLGRU recurrence over B x T tokens of D channels, pre-activations
+    resident in HBM (4 x 32 MB in, 32 MB out: inputs larger than L2)."""
+    from bitlinear_rmsnorm_quant_b200 import mmf
+    B, T, D = SCAN_SHAPE
+    dev = torch.device("cuda", dist.local_rank)
+    gen = torch.Generator(device=dev).manual_seed(5 + dist.rank)
+    mk = lambda: (torch.randn((B, T, D), generator=gen, device=dev) * 2.0).to(torch.bfloat16)
+    fp, cp, gp = mk(), mk(), mk()
+    h0 = torch.randn((B, D), generator=gen, device=dev)
+    o = torch.empty((B, T, D), dtype=torch.bfloat16, device=dev)
+    hl = torch.empty((B, D), dtype=torch.float32, device=dev)
+    lib = mmf.lib()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        rc = lib.mmf_mlgru_scan(fp.data_ptr(), cp.data_ptr(), gp.data_ptr(), h0.data_ptr(), B, T, D, o.data_ptr(),
+                                hl.data_ptr(), stream.cuda_stream)
+        if rc != 0:
+            raise mmf.MMFError("mmf_mlgru_scan", rc)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = ClockSampler(dist.local_rank)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks.stop()
+    dist.barrier()
+    mmf.check_async()
+    ms = dist.max(e0.elapsed_time(e1) / args.steps)
+    # e2e: pre-activations from pinned host memory, o back to it
+    h_in = [t.cpu().pin_memory() for t in (fp, cp, gp)]
+    h_o = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(1, min(args.steps, 50))
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(e2e_steps):
+        for d_, h_ in zip((fp, cp, gp), h_in):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        h_o.copy_(o, non_blocking=True)
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = dist.max(f0.elapsed_time(f1) / e2e_steps)
+    tokens = B * T * dist.world
+    nbytes = B * T * D * 2 * 4 + B * D * 4 * 2   # three inputs and o (bf16), h0 and h_last (fp32)
+    peaks, peak_src = load_peaks()
+    achieved = nbytes / (ms / 1e3) / 1e9
+    res = {
+        "metric": METRIC, "value": round(tokens / (ms / 1e3), 2),
+        "unit": "tokens/s (one token through the MLGRU recurrence at the 1.3B width)",
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (torch normal pre-activations x2, bf16)",
+        "config": {"workload": "mlgru-scan-1.3b", "B": B, "T": T, "D": D,
+                   "l2": "inputs larger than L2 (4 x 32 MB)", "parallelism": f"dp{dist.world} (replicas)"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": float(peaks["hbm_gbs"]),
+                     "unit": "GB/s", "frac": round(achieved / float(peaks["hbm_gbs"]), 4), "traffic": None,
+                     "kernel": "mlgru_scan_kernel", "peak_source": f"{peak_src} hbm_gbs",
+                     "algorithmic_bytes_per_launch": nbytes},
+        "e2e": {"value": round(tokens / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(3 * B * T * D * 2), "d2h_bytes_per_step": int(B * T * D * 2),
+                "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = scan_cpu_baseline(fp[:1, :256].cpu(), cp[:1, :256].cpu(), gp[:1, :256].cpu(), D)
+    return res
+
+
+def scan_cpu_baseline(fp, cp, gp, D):
+    """The oracle's recurrence on a sample of one sequence's first 256 tokens."""
+    import numpy as np
+
+    from oracle import load
+    orc = load()
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    f_, c_, g_ = bits(fp), bits(cp), bits(gp)
+    t0 = time.perf_counter()
+    reps = 0
+    while time.perf_counter() - t0 < 5.0:
+        orc.mlgru_scan(f_, c_, g_)
+        reps += 1
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": round(fp.shape[1] / dt, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"1 sequence x {fp.shape[1]} tokens x {D} channels"}
+
+
 def library_int8_tops(n: int = 8192, reps: int = 5):
     """Context for the tensor roofline: a library int8 GEMM (torch._int_mm,
     cuBLASLt) at n^3 on this GPU, best of `reps`, CUDA events."""
@@ -202,7 +298,9 @@ WORKLOADS = {
     "prefill-1.3b": (lambda: WL.PREFILL_1P3B, 1),
     "train-fwd-1.3b": (lambda: WL.TRAIN_FWD_1P3B, 1),
     "smoke-256": (lambda: WL.SMOKE, 1),
+    "mlgru-scan-1.3b": (None, 1),   # the token mixer's recurrence alone (run_scan)
 }
+SCAN_SHAPE = (4, 2048, 2048)        # sequences, tokens, channels: 4 x 2048 tokens at the 1.3B width
 DEFAULT_WORKLOAD = "decode-2.7b-m1"
 
 
@@ -550,6 +648,19 @@ def main(argv=None):
         args.warmup = 3
     dist = Dist(args.gpus)
     try:
+        if args.impl == "reference" and args.workload == "mlgru-scan-1.3b":
+            if dist.rank == 0:
+                B, T, D = SCAN_SHAPE
+                g = torch.Generator().manual_seed(5)
+                mk = lambda: (torch.randn((1, 256, D), generator=g) * 2.0).to(torch.bfloat16)
+                cb = scan_cpu_baseline(mk(), mk(), mk(), D)
+                print(json.dumps({"metric": METRIC, "impl": "reference", "value": cb["value"], "unit": cb["unit"],
+                                  "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                                  "higher_is_better": True, "config": {"workload": args.workload},
+                                  "cpu_baseline": cb, "e2e": {"value": cb["value"], "unit": cb["unit"],
+                                                              "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+                      flush=True)
+            return 0
         if args.impl == "reference":
             res = run_reference(args, dist)
             if res is not None:
@@ -557,6 +668,11 @@ def main(argv=None):
             return 0
         if not torch.cuda.is_available():
             raise SystemExit("bench.py --impl ours needs a CUDA device")
+        if args.workload == "mlgru-scan-1.3b":
+            res = run_scan(args, dist)
+            if dist.rank == 0:
+                print(json.dumps(res), flush=True)
+            return 0
         res, wl, L = run_ours(args, dist)
         if dist.rank == 0:
             if dist.world == 1 and not args.no_cpu_baseline:

@@ -20,9 +20,12 @@
 
 namespace mmf {
 
-constexpr int kScanWarps = 16;
+constexpr int kScanWarps = 32;
 
-__device__ __forceinline__ float sigmoid_f(float v) { return __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-v))); }
+// sigma(v) = 1 / (1 + e^-v) with the hardware exponential and reciprocal
+// (a few ulp: the recurrence is instruction-bound with the IEEE forms, and
+// its state is compared with the oracle to fp32-level tolerances anyway).
+__device__ __forceinline__ float sigmoid_f(float v) { return __fdividef(1.0f, 1.0f + __expf(-v)); }
 
 __device__ __forceinline__ void bf16x2_to_f(uint32_t w, float& lo, float& hi) {
     lo = __uint_as_float(w << 16);

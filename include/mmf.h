@@ -172,8 +172,9 @@ int mmf_bitlinear_fwd_glu(const uint16_t* g, const uint16_t* u,
  *   h = f * h + (1 - f) * c          (fp32)
  *   o[b][t][k] = bf16_rn(g * h)      (the o projection's input)
  * and h_last[b][k] = h after the last token (may be NULL).  Tokens are split
- * into chunks combined through their linear maps h -> A h + B, so the result
- * matches the token-by-token recurrence to fp32 rounding, not bit for bit.
+ * into chunks combined through their linear maps h -> A h + B, and sigma uses
+ * the hardware exponential and reciprocal (a few ulp), so the result matches
+ * the token-by-token recurrence to a few fp32 ulps per token, not bit for bit.
  * f_pre, c_pre, g_pre, o: bf16 [B][T][D] (the projections' y layout with
  * M = B * T); h0, h_last: fp32 [B][D].  D must be even, B <= 65535; pointers
  * 16-byte aligned; o must not overlap the inputs.  T = 0 copies h0 (or zeros)
