@@ -215,19 +215,21 @@ __global__ void __launch_bounds__(kQuantCtaWarps * 32) rmsnorm_quant_kernel(cons
 // of the definition never changes a code.  Four bytes are packed with byte
 // permutes and summed with one DP4A.
 constexpr int kQuantStreamWarps = 8;
-constexpr int kMaxQuantStreamK = 7168;  // 8 warps x 2 rows of bf16 within the 227 KB of one CTA
+constexpr int kMaxQuantStreamK = 6400;  // gamma + 8 warps x 2 rows of bf16 within the 227 KB of one CTA
 
 __host__ __device__ inline size_t quant_stream_smem(int K) {
-    return static_cast<size_t>(kQuantStreamWarps) * 2 * 2 * static_cast<size_t>(K);
+    return static_cast<size_t>(4) * K + static_cast<size_t>(kQuantStreamWarps) * 2 * 2 * static_cast<size_t>(K);
 }
 
 __global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ gamma, float eps, int K, int64_t M,
     int8_t* __restrict__ q, float* __restrict__ absmax, int* __restrict__ qsum) {
-    extern __shared__ __align__(128) uint4 xs_all[];  // [warp][2 buffers][K/8 chunks]
+    extern __shared__ __align__(128) uint4 smem_q[];  // gamma fp32 [K], then [warp][2 buffers][K/8 chunks]
     __shared__ __align__(8) uint64_t row_bar[kQuantStreamWarps][2];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int C = K >> 3;
+    float4* gamma_s = reinterpret_cast<float4*>(smem_q);
+    uint4* xs_all = smem_q + (K >> 2);
     const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
     const int64_t gw = static_cast<int64_t>(blockIdx.x) * kQuantStreamWarps + warp;
     const int64_t TW = static_cast<int64_t>(gridDim.x) * kQuantStreamWarps;
@@ -237,7 +239,9 @@ __global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_k
         mbar_init(&row_bar[warp][1], 1);
         mbar_fence_init();
     }
-    __syncwarp();
+    // gamma once per CTA into shared memory (read by every row, twice)
+    for (int j = threadIdx.x; j < (K >> 2); j += blockDim.x) gamma_s[j] = __ldg(reinterpret_cast<const float4*>(gamma) + j);
+    __syncthreads();
     pdl_wait();  // x may come from the previous kernel (no-op unless launched as a dependent)
     pdl_launch_dependents();
     auto issue = [&](int64_t m, int b) {
@@ -251,7 +255,7 @@ __global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_k
         }
     };
     if (gw < M) issue(gw, 0);
-    const float4* g4 = reinterpret_cast<const float4*>(gamma);
+    const float4* g4 = gamma_s;
     int i = 0;
     for (int64_t m = gw; m < M; m += TW, ++i) {
         const int b = i & 1;
@@ -281,7 +285,7 @@ __global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_k
         for (int c = lane; c < C; c += 32) {
             float f[8];
             unpack_bf16x8(xs[c], f);
-            const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
+            const float4 ga = g4[2 * c], gb = g4[2 * c + 1];
             const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
 #pragma unroll
             for (int k = 0; k < 8; ++k)
@@ -297,7 +301,7 @@ __global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_k
         for (int c = lane; c < C; c += 32) {
             float f[8];
             unpack_bf16x8(xs[c], f);
-            const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
+            const float4 ga = g4[2 * c], gb = g4[2 * c + 1];
             const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
             uint32_t cb[8];  // codes in the low bytes
 #pragma unroll
