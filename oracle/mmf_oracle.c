@@ -228,6 +228,60 @@ void orc_mlgru_scan(const uint16_t* f_pre, const uint16_t* c_pre, const uint16_t
     }
 }
 
+int orc_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma, float eps,
+                      const int8_t* wt, float beta, int64_t M, int64_t K, int64_t N,
+                      uint16_t* dx, float* dgamma, float* dW) {
+    int8_t* q = (int8_t*)malloc((size_t)(M * K > 0 ? M * K : 1));
+    float* a = (float*)malloc(sizeof(float) * (size_t)(M > 0 ? M : 1));
+    double* dr = (double*)malloc(sizeof(double) * (size_t)(M * K > 0 ? M * K : 1));
+    double* dg = (double*)calloc((size_t)(K > 0 ? K : 1), sizeof(double));
+    if (!q || !a || !dr || !dg) {
+        free(q);
+        free(a);
+        free(dr);
+        free(dg);
+        return -1;
+    }
+    orc_rmsnorm_quant(x, gamma, eps, M, K, q, a);
+    /* dr = dy . W_q */
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t n = 0; n < N; ++n) s += (double)orc_bf16_to_f32(dy[m * N + n]) * (double)wt[n * K + k];
+            dr[m * K + k] = s * (double)beta;
+        }
+    /* dW = dy^T . x_q */
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t m = 0; m < M; ++m)
+                s += (double)orc_bf16_to_f32(dy[m * N + n]) * ((double)q[m * K + k] * ((double)a[m] / 127.0));
+            dW[n * K + k] = (float)s;
+        }
+    /* RMSNorm backward */
+    for (int64_t m = 0; m < M; ++m) {
+        double s2 = 0.0, dot = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const double xv = (double)orc_bf16_to_f32(x[m * K + k]);
+            s2 += xv * xv;
+            dot += (double)gamma[k] * dr[m * K + k] * xv;
+        }
+        const double inv = 1.0 / sqrt(s2 / (double)K + (double)eps);
+        for (int64_t k = 0; k < K; ++k) {
+            const double xv = (double)orc_bf16_to_f32(x[m * K + k]);
+            const double g = inv * (double)gamma[k] * dr[m * K + k] - xv * inv * inv * inv * dot / (double)K;
+            dx[m * K + k] = orc_f64_to_bf16(g);
+            dg[k] += dr[m * K + k] * xv * inv;
+        }
+    }
+    for (int64_t k = 0; k < K; ++k) dgamma[k] = (float)dg[k];
+    free(q);
+    free(a);
+    free(dr);
+    free(dg);
+    return 0;
+}
+
 int orc_bitlinear(const uint16_t* x, const float* gamma, float eps,
                   const float* W, float eps_w, int64_t M, int64_t K, int64_t N,
                   uint16_t* y, float* beta_out) {

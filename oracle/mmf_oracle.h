@@ -113,6 +113,27 @@ void orc_glu_gate(const uint16_t* g, const uint16_t* u, int64_t n, uint16_t* p);
 void orc_mlgru_scan(const uint16_t* f_pre, const uint16_t* c_pre, const uint16_t* g_pre,
                     const float* h0, int64_t B, int64_t T, int64_t D, uint16_t* o, float* h_last);
 
+/* Backward of the fused BitLinear layer with the straight-through estimator
+ * (ld246.com, section "训练与优化：新的策略": the non-differentiable ternary
+ * weights and quantisation are back-propagated with a surrogate gradient, the
+ * straight-through estimator, read as passing gradients through the
+ * quantisers unchanged).  Forward: r = RMSNorm(x) *
+ * gamma, x_q = q * (absmax / 127) (the quantised r), W_q = w~ * beta,
+ * y = x_q . W_q^T.  With both quantisers taken as the identity:
+ *   dr[m][k]  = sum_n dy[m][n] * W_q[n][k]
+ *   dW[n][k]  = sum_m dy[m][n] * x_q[m][k]
+ *   dgamma[k] = sum_m dr[m][k] * x[m][k] * inv_m
+ *   dx[m][k]  = inv_m * gamma[k] * dr[m][k]
+ *               - x[m][k] * inv_m^3 * (sum_j gamma[j] dr[m][j] x[m][j]) / K
+ * with inv_m = 1 / sqrt(sum_k x^2 / K + eps); all in fp64, dx rounded to
+ * bf16.  q and absmax are the forward's (orc_rmsnorm_quant).
+ * dy bf16 [M][N]; x bf16 [M][K]; wt int8 [N][K]; dx bf16 [M][K];
+ * dgamma fp32 [K]; dW fp32 [N][K].  Returns 0, or -1 if scratch allocation
+ * failed. */
+int orc_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma, float eps,
+                      const int8_t* wt, float beta, int64_t M, int64_t K, int64_t N,
+                      uint16_t* dx, float* dgamma, float* dW);
+
 /* Number of OpenMP threads orc_ternary_acc uses (1 when built without OpenMP). */
 int orc_num_threads(void);
 

@@ -49,6 +49,8 @@ class Oracle:
         lib.orc_glu_gate.restype = None
         lib.orc_mlgru_scan.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]
         lib.orc_mlgru_scan.restype = None
+        lib.orc_bitlinear_bwd.argtypes = [_P, _P, _P, _F, _P, _F, _I64, _I64, _I64, _P, _P, _P]
+        lib.orc_bitlinear_bwd.restype = C.c_int
         lib.orc_num_threads.argtypes = []
         lib.orc_num_threads.restype = C.c_int
         self.lib = lib
@@ -141,6 +143,22 @@ class Oracle:
             h0p = _ptr(h0)
         self.lib.orc_mlgru_scan(_ptr(f_bits), _ptr(c_bits), _ptr(g_bits), h0p, B, T, D, _ptr(o), _ptr(h_last))
         return o, h_last
+
+    def bitlinear_bwd(self, dy_bits, x_bits, gamma, eps, wt, beta):
+        """-> (dx bf16 bits [M, K], dgamma fp32 [K], dW fp32 [N, K]) under the straight-through estimator."""
+        dy_bits = np.ascontiguousarray(dy_bits, dtype=np.uint16)
+        x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        gamma = np.ascontiguousarray(gamma, dtype=np.float32)
+        wt = np.ascontiguousarray(wt, dtype=np.int8)
+        M, K = x_bits.shape
+        N = wt.shape[0]
+        dx = np.empty((M, K), dtype=np.uint16)
+        dg = np.empty(K, dtype=np.float32)
+        dW = np.empty((N, K), dtype=np.float32)
+        if self.lib.orc_bitlinear_bwd(_ptr(dy_bits), _ptr(x_bits), _ptr(gamma), eps, _ptr(wt), float(beta),
+                                      M, K, N, _ptr(dx), _ptr(dg), _ptr(dW)) != 0:
+            raise MemoryError("oracle allocation failed")
+        return dx, dg, dW
 
     def bitlinear(self, x_bits, gamma, eps, W, eps_w):
         x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)

@@ -23,6 +23,8 @@ quantisers' error bounds and hand-worked tiny cases):
                      exact zeros, SiLU(v) - SiLU(-v) = v, saturation
   MLGRU recurrence   closed form for constant gates and inputs, forgetting and
                      keeping limits, continuation across calls, independence
+  STE backward       central differences of the surrogate forward (dx, dgamma),
+                     matmul with the quantised activations (dW), linearity in dy
 """
 from __future__ import annotations
 
@@ -386,6 +388,53 @@ def check_mlgru_scan(orc):
     assert np.array_equal(o_all[1:], o_b1)
 
 
+def check_bitlinear_bwd(orc):
+    """The straight-through backward against central differences of the
+    surrogate forward y = (RMSNorm(x) gamma) . W_q^T in fp64 (x and gamma
+    perturbed, quantisers absent), dW against the matmul with the quantised
+    activations, zeros for dy = 0 and exact doubling for 2 dy."""
+    rng = np.random.default_rng(51)
+    M, K, N, eps = 3, 16, 5, 1e-6
+    xb = _torch_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    dyb = _torch_bf16_bits(rng.standard_normal((M, N)).astype(np.float32))
+    g = (1.0 + 0.1 * rng.standard_normal(K)).astype(np.float32)
+    wt = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    beta = np.float32(0.0175)
+    dx, dg, dW = orc.bitlinear_bwd(dyb, xb, g, eps, wt, beta)
+    xv, dy = _bf16_bits_to_f64(xb), _bf16_bits_to_f64(dyb)
+    Wq = wt.astype(np.float64) * float(beta)
+
+    def loss(x, gamma):
+        inv = 1.0 / np.sqrt((x * x).mean(axis=1, keepdims=True) + eps)
+        return float(((x * inv * gamma) @ Wq.T * dy).sum())
+
+    h = 1e-6
+    num_dx = np.zeros((M, K))
+    num_dg = np.zeros(K)
+    for m in range(M):
+        for k in range(K):
+            e = np.zeros((M, K))
+            e[m, k] = h
+            num_dx[m, k] = (loss(xv + e, g.astype(np.float64)) - loss(xv - e, g.astype(np.float64))) / (2 * h)
+    for k in range(K):
+        e = np.zeros(K)
+        e[k] = h
+        num_dg[k] = (loss(xv, g + e) - loss(xv, g - e)) / (2 * h)
+    dxv = _bf16_bits_to_f64(dx)
+    assert np.allclose(dxv, num_dx, rtol=2.0 ** -7, atol=1e-6)
+    assert np.allclose(dg, num_dg, rtol=1e-5, atol=1e-6)
+    q, a = orc.rmsnorm_quant(xb, g, eps)
+    xq = q.astype(np.float64) * (a.astype(np.float64)[:, None] / 127.0)
+    assert np.allclose(dW, dy.T @ xq, rtol=1e-6, atol=1e-9)
+    zero = np.zeros_like(dyb)
+    dx0, dg0, dW0 = orc.bitlinear_bwd(zero, xb, g, eps, wt, beta)
+    assert (_bf16_bits_to_f64(dx0) == 0).all() and (dg0 == 0).all() and (dW0 == 0).all()
+    dy2 = _bits_of(2.0 * _bf16_bits_to_f64(dyb).astype(np.float32))
+    dx2, dg2, dW2 = orc.bitlinear_bwd(dy2, xb, g, eps, wt, beta)
+    assert np.array_equal(_bf16_bits_to_f64(dx2), 2.0 * dxv) and np.array_equal(dg2, 2.0 * dg)
+    assert np.array_equal(dW2, 2.0 * dW)
+
+
 ALL_CHECKS = [
     check_bf16_rounding,
     check_absmean_worked_ties,
@@ -403,4 +452,5 @@ ALL_CHECKS = [
     check_layer_bound,
     check_glu_gate,
     check_mlgru_scan,
+    check_bitlinear_bwd,
 ]

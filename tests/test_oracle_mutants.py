@@ -41,6 +41,10 @@ MUTANTS = [
     ("forget-swapped", "h = f * h + (1.0f - f) * c;", "h = (1.0f - f) * h + f * c;"),
     ("no-output-gate", "o[i] = orc_f64_to_bf16((double)(g * h));", "o[i] = orc_f64_to_bf16((double)h);"),
     ("silu-as-sigmoid", "const float c = cv * orc_sigmoid(cv);", "const float c = orc_sigmoid(cv);"),
+    ("bwd-missing-norm-term", "- xv * inv * inv * inv * dot / (double)K;", "- 0.0 * dot;"),
+    ("bwd-dW-unscaled", "((double)q[m * K + k] * ((double)a[m] / 127.0));", "((double)q[m * K + k]);"),
+    ("bwd-dr-transposed-w", "s += (double)orc_bf16_to_f32(dy[m * N + n]) * (double)wt[n * K + k];",
+     "s += (double)orc_bf16_to_f32(dy[m * N + n]) * (double)wt[(k % N) * K + (n % K)];"),
 ]
 
 
