@@ -145,6 +145,74 @@ def run_scan(args, dist):
     return res
 
 
+def run_bwd(args, dist):
+    """Backward of the three prefill projections at the 1.3B width (M = 8192):
+    two bf16 GEMMs each (dr and dW) plus the straight-through operand
+    preparation and the RMSNorm backward."""
+    from bitlinear_rmsnorm_quant_b200 import mmf
+    wl = WL.PREFILL_1P3B
+    M = wl.M
+    dev = torch.device("cuda", dist.local_rank)
+    lib = mmf.lib()
+    stream = torch.cuda.current_stream()
+    items = []
+    for j, p in enumerate(wl.projections):
+        x = I.activations(wl.seed, M, p.K, index=p.input_index, device=dev)
+        g = I.gamma(wl.seed, p.K, index=p.input_index, device=dev)
+        W = I.latent_weights(wl.seed, p.N, p.K, index=j, device=dev)
+        packed, scale = mmf.pack_ternary(W, wl.eps_w)
+        del W
+        dy = I.activations(wl.seed, M, p.N, index=32 + j, device=dev)
+        dx = torch.empty((M, p.K), dtype=torch.bfloat16, device=dev)
+        dg = torch.empty(p.K, dtype=torch.float32, device=dev)
+        dW = torch.empty((p.N, p.K), dtype=torch.float32, device=dev)
+        ws = torch.empty(int(lib.mmf_bwd_workspace_bytes(M, p.K, p.N)), dtype=torch.uint8, device=dev)
+        items.append((p, x, g, packed, scale, dy, dx, dg, dW, ws))
+
+    def step():
+        for p, x, g, packed, scale, dy, dx, dg, dW, ws in items:
+            rc = lib.mmf_bitlinear_bwd(dy.data_ptr(), x.data_ptr(), g.data_ptr(), wl.eps, packed.data_ptr(),
+                                       scale.data_ptr(), M, p.K, p.N, dx.data_ptr(), dg.data_ptr(), dW.data_ptr(),
+                                       ws.data_ptr(), ws.numel(), stream.cuda_stream)
+            if rc != 0:
+                raise mmf.MMFError("mmf_bitlinear_bwd", rc)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = ClockSampler(dist.local_rank)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks.stop()
+    dist.barrier()
+    mmf.check_async()
+    ms = dist.max(e0.elapsed_time(e1) / args.steps)
+    flops = sum(2 * 2 * M * p.N * p.K for p in wl.projections)
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    return {
+        "metric": METRIC, "value": round(M * dist.world / (ms / 1e3), 2),
+        "unit": "tokens/s (one token back through the three prefill projections)",
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64/Box-Muller)",
+        "config": {"workload": "bwd-prefill-1.3b", "M": M, "projections": [f"{p.K}->{p.N}" for p in wl.projections],
+                   "parallelism": f"dp{dist.world} (replicas)"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None, "kernel": "cuBLAS bf16 GEMMs + own kernels",
+                     "peak_source": f"{peak_src} bf16_tflops", "algorithmic_flops_per_step": flops},
+        "gpu_launches": 7 * len(items) * args.steps,   # ours; cuBLAS adds its own GEMM kernels
+        "clocks": clocks.summary(),
+    }
+
+
 def scan_cpu_baseline(fp, cp, gp, D):
     """The oracle's recurrence on a sample of one sequence's first 256 tokens."""
     import numpy as np
@@ -299,6 +367,7 @@ WORKLOADS = {
     "train-fwd-1.3b": (lambda: WL.TRAIN_FWD_1P3B, 1),
     "smoke-256": (lambda: WL.SMOKE, 1),
     "mlgru-scan-1.3b": (None, 1),   # the token mixer's recurrence alone (run_scan)
+    "bwd-prefill-1.3b": (None, 1),  # straight-through backward of the prefill projections (run_bwd)
 }
 SCAN_SHAPE = (4, 2048, 2048)        # sequences, tokens, channels: 4 x 2048 tokens at the 1.3B width
 DEFAULT_WORKLOAD = "decode-2.7b-m1"
@@ -661,6 +730,11 @@ def main(argv=None):
                                                               "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
                       flush=True)
             return 0
+        if args.impl == "reference" and WORKLOADS[args.workload][0] is None:
+            if dist.rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable":
+                                  f"no oracle arm for --workload {args.workload}; use the default workload"}))
+            return 0
         if args.impl == "reference":
             res = run_reference(args, dist)
             if res is not None:
@@ -668,8 +742,8 @@ def main(argv=None):
             return 0
         if not torch.cuda.is_available():
             raise SystemExit("bench.py --impl ours needs a CUDA device")
-        if args.workload == "mlgru-scan-1.3b":
-            res = run_scan(args, dist)
+        if args.workload in ("mlgru-scan-1.3b", "bwd-prefill-1.3b"):
+            res = run_scan(args, dist) if args.workload == "mlgru-scan-1.3b" else run_bwd(args, dist)
             if dist.rank == 0:
                 print(json.dumps(res), flush=True)
             return 0

@@ -3,7 +3,9 @@
 // the headers included below; this is the only translation unit.
 #include "mmf.h"
 
+#include <cublas_v2.h>
 #include <cudaTypedefs.h>
+#include <dlfcn.h>
 
 #include <mutex>
 #include <utility>
@@ -15,6 +17,7 @@
 #include "pack.cuh"
 #include "quant.cuh"
 #include "scan.cuh"
+#include "bwd.cuh"
 
 namespace {
 
@@ -27,7 +30,21 @@ constexpr int64_t kMaxK = 65536;  // the quantiser stages one bf16 row (2K bytes
 struct DeviceState {
     bool ready = false;
     int num_sms = 0;
+    cublasHandle_t cublas = nullptr;  // backward only, created on first use
 };
+
+// cuBLAS serves the backward's two plain bf16 GEMMs only; it is opened on the
+// first backward call, so the forward path never depends on it.
+using CublasGemmExFn = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int,
+                                          const void*, const void*, cudaDataType, int, const void*, cudaDataType, int,
+                                          const void*, void*, cudaDataType, int, cublasComputeType_t, cublasGemmAlgo_t);
+struct CublasApi {
+    decltype(&cublasCreate_v2) create = nullptr;
+    decltype(&cublasSetStream_v2) set_stream = nullptr;
+    CublasGemmExFn gemm = nullptr;
+    bool tried = false;
+};
+CublasApi g_cublas;
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -464,6 +481,103 @@ int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps, const ui
     pr.y = y;
     pr.N = N;
     return fwd_impl(x, gamma, eps, M, K, &pr, 1, workspace, 0u, static_cast<cudaStream_t>(stream), dev);
+}
+
+size_t mmf_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+    if (check_shape(M, K, N) != MMF_OK) return 0;
+    const size_t m = static_cast<size_t>(M), k = static_cast<size_t>(K), n = static_cast<size_t>(N);
+    const size_t chunks = (m + kDgammaRows - 1) / kDgammaRows;
+    return align256(m * k) + 3 * align256(4 * m) + align256(2 * n * k) + align256(2 * m * n) + align256(2 * m * k) +
+           align256(4 * m * k) + align256(8 * chunks * k);
+}
+
+int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma, float eps, const uint32_t* packed,
+                      const float* scale, int64_t M, int64_t K, int64_t N, uint16_t* dx, float* dgamma, float* dW,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    if (!(eps >= 0.0f) || eps > 1e30f) return MMF_ERR_INVALID_ARG;
+    mmf_status st = check_shape(M, K, N);
+    if (st != MMF_OK) return st;
+    // 32-bit GEMM sizes; the dgamma row chunks on grid.y
+    if (M > 65535L * kDgammaRows || N * M > kMaxDim || M * K > kMaxDim) return MMF_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 && N == 0) return MMF_OK;
+    if (!dy || !x || !gamma || !packed || !scale || !dx || !dgamma || !dW || !workspace)
+        return MMF_ERR_INVALID_ARG;
+    if (!aligned16(dy) || !aligned16(x) || !aligned16(gamma) || !aligned16(packed) || !aligned16(scale) ||
+        !aligned16(dx) || !aligned16(dgamma) || !aligned16(dW) || !aligned16(workspace))
+        return MMF_ERR_MISALIGNED;
+    if (workspace_bytes < mmf_bwd_workspace_bytes(M, K, N)) return MMF_ERR_WORKSPACE;
+    DeviceState* dev;
+    if ((st = device_state(&dev)) != MMF_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!g_cublas.tried) {
+            g_cublas.tried = true;
+            void* h = dlopen("libcublas.so.12", RTLD_NOW | RTLD_LOCAL);
+            if (h) {
+                g_cublas.create = reinterpret_cast<decltype(&cublasCreate_v2)>(dlsym(h, "cublasCreate_v2"));
+                g_cublas.set_stream = reinterpret_cast<decltype(&cublasSetStream_v2)>(dlsym(h, "cublasSetStream_v2"));
+                g_cublas.gemm = reinterpret_cast<CublasGemmExFn>(dlsym(h, "cublasGemmEx"));
+            }
+        }
+        if (!g_cublas.create || !g_cublas.set_stream || !g_cublas.gemm) return MMF_ERR_CUDA;
+        if (!dev->cublas && g_cublas.create(&dev->cublas) != CUBLAS_STATUS_SUCCESS) return MMF_ERR_CUDA;
+    }
+    // workspace: q, absmax, qsum, inv, w~ (bf16), dy * absmax / 127 (bf16), q (bf16), dr (fp32)
+    uint8_t* b = static_cast<uint8_t*>(workspace);
+    const size_t m = static_cast<size_t>(M), k = static_cast<size_t>(K), n = static_cast<size_t>(N);
+    int8_t* q = reinterpret_cast<int8_t*>(b);
+    b += align256(m * k);
+    float* absmax = reinterpret_cast<float*>(b);
+    b += align256(4 * m);
+    int* qsum = reinterpret_cast<int*>(b);
+    b += align256(4 * m);
+    float* inv = reinterpret_cast<float*>(b);
+    b += align256(4 * m);
+    uint16_t* wb = reinterpret_cast<uint16_t*>(b);
+    b += align256(2 * n * k);
+    uint16_t* dys = reinterpret_cast<uint16_t*>(b);
+    b += align256(2 * m * n);
+    uint16_t* qb = reinterpret_cast<uint16_t*>(b);
+    b += align256(2 * m * k);
+    float* dr = reinterpret_cast<float*>(b);
+    b += align256(4 * m * k);
+    double* part = reinterpret_cast<double*>(b);
+    const int chunks = static_cast<int>((M + kDgammaRows - 1) / kDgammaRows);
+
+    if (M > 0 && (st = launch_quant(x, gamma, eps, M, K, q, absmax, qsum, s, false, dev->num_sms)) != MMF_OK) return st;
+    const auto blocks = [](int64_t count) { return dim3(static_cast<unsigned>((count + kBwdThreads - 1) / kBwdThreads)); };
+    if (N > 0 && (st = launch(unpack_ternary_bf16_kernel, blocks(N * K / 16), dim3(kBwdThreads), 0, s, false, packed,
+                              N * K / 16, wb)) != MMF_OK)
+        return st;
+    if (M > 0 && N > 0 &&
+        (st = launch(scale_dy_kernel, blocks(M * N), dim3(kBwdThreads), 0, s, false, dy, absmax, M, N, dys)) != MMF_OK)
+        return st;
+    if (M > 0 && (st = launch(codes_bf16_kernel, blocks(M * K), dim3(kBwdThreads), 0, s, false, q, M * K, qb)) != MMF_OK)
+        return st;
+    if (g_cublas.set_stream(dev->cublas, s) != CUBLAS_STATUS_SUCCESS) return MMF_ERR_CUDA;
+    const float one = 1.0f, zero = 0.0f;
+    // dr[M][K] = dy[M][N] . w~[N][K]   (column-major: dr^T = w~^T dy^T)
+    if (M > 0 && g_cublas.gemm(dev->cublas, CUBLAS_OP_N, CUBLAS_OP_N, static_cast<int>(K), static_cast<int>(M),
+                               static_cast<int>(N), &one, wb, CUDA_R_16BF, static_cast<int>(K), dy, CUDA_R_16BF,
+                               static_cast<int>(N), &zero, dr, CUDA_R_32F, static_cast<int>(K), CUBLAS_COMPUTE_32F,
+                               CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+        return MMF_ERR_CUDA;
+    // dW[N][K] = dys^T[N][M] . q[M][K]   (column-major: dW^T = q^T dys)
+    if (N > 0 && g_cublas.gemm(dev->cublas, CUBLAS_OP_N, CUBLAS_OP_T, static_cast<int>(K), static_cast<int>(N),
+                               static_cast<int>(M), &one, qb, CUDA_R_16BF, static_cast<int>(K), dys, CUDA_R_16BF,
+                               static_cast<int>(N), &zero, dW, CUDA_R_32F, static_cast<int>(K), CUBLAS_COMPUTE_32F,
+                               CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+        return MMF_ERR_CUDA;
+    if (M > 0 && (st = launch(rmsnorm_bwd_kernel, dim3(static_cast<unsigned>(M)), dim3(kBwdThreads), 0, s, false, x,
+                              gamma, static_cast<const float*>(dr), scale, eps, static_cast<int>(K), dx, inv)) != MMF_OK)
+        return st;
+    if (M > 0 && (st = launch(dgamma_partial_kernel, dim3(blocks(K).x, static_cast<unsigned>(chunks)), dim3(kBwdThreads),
+                              0, s, false, x, static_cast<const float*>(dr), static_cast<const float*>(inv), M,
+                              static_cast<int>(K), part)) != MMF_OK)
+        return st;
+    return launch(dgamma_final_kernel, blocks(K), dim3(kBwdThreads), 0, s, false, static_cast<const double*>(part), chunks,
+                  static_cast<int>(K), scale, dgamma);
 }
 
 int mmf_mlgru_scan(const uint16_t* f_pre, const uint16_t* c_pre, const uint16_t* g_pre, const float* h0, int64_t B,

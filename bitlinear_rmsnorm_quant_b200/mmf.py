@@ -42,6 +42,8 @@ SIGNATURES = {
     "mmf_bitlinear_fwd": (_INT, [_P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "mmf_bitlinear_fwd_glu": (_INT, [_P, _P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, C.c_uint, _P]),
     "mmf_mlgru_scan": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P]),
+    "mmf_bwd_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "mmf_bitlinear_bwd": (_INT, [_P, _P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
     "mmf_bitlinear_fwd_group": (_INT, [_P, _P, _F, _I64, _I64, _P, _INT, _P, _SZ, C.c_uint, _P]),
     "mmf_bitlinear_fwd_noalloc": (_INT, [_P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _P]),
     "mmf_hbm_copy": (_INT, [_P, _P, _SZ, _P]),
@@ -220,6 +222,24 @@ def mlgru_scan(f_pre: torch.Tensor, c_pre: torch.Tensor, g_pre: torch.Tensor, h0
                                h0.data_ptr() if h0 is not None else None, B, T, D, o.data_ptr(), hl.data_ptr(),
                                _stream(stream)), "mmf_mlgru_scan")
     return o, hl
+
+
+def bitlinear_bwd(dy: torch.Tensor, x: torch.Tensor, gamma: torch.Tensor, packed: torch.Tensor,
+                  scale: torch.Tensor, eps: float = 1e-6, stream=None):
+    """Straight-through backward: bf16 dy[M, N], x[M, K] -> (bf16 dx[M, K], fp32 dgamma[K], fp32 dW[N, K])."""
+    _dev(dy, torch.bfloat16, "dy")
+    _dev(x, torch.bfloat16, "x")
+    M, K = x.shape
+    N = dy.shape[1]
+    dx = torch.empty((M, K), dtype=torch.bfloat16, device=x.device)
+    dg = torch.empty(K, dtype=torch.float32, device=x.device)
+    dW = torch.empty((N, K), dtype=torch.float32, device=x.device)
+    n = int(lib().mmf_bwd_workspace_bytes(M, K, N))
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=x.device)
+    check(lib().mmf_bitlinear_bwd(dy.data_ptr(), x.data_ptr(), gamma.data_ptr(), eps, packed.data_ptr(),
+                                  scale.data_ptr(), M, K, N, dx.data_ptr(), dg.data_ptr(), dW.data_ptr(),
+                                  ws.data_ptr(), ws.numel(), _stream(stream)), "mmf_bitlinear_bwd")
+    return dx, dg, dW
 
 
 def bitlinear_fwd_group(x: torch.Tensor, gamma: torch.Tensor, weights, eps: float = 1e-6, workspace=None,

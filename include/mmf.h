@@ -184,6 +184,30 @@ int mmf_mlgru_scan(const uint16_t* f_pre, const uint16_t* c_pre,
                    const uint16_t* g_pre, const float* h0, int64_t B, int64_t T,
                    int64_t D, uint16_t* o, float* h_last, void* stream);
 
+/*
+ * mmf_bitlinear_bwd -- backward of mmf_bitlinear_fwd with the straight-through
+ * estimator (ld246.com, section "训练与优化：新的策略": the non-differentiable
+ * ternary weights and quantisation are back-propagated with a surrogate
+ * gradient, read as passing gradients through both quantisers unchanged).
+ * With x_q = q * (absmax / 127) (the forward's codes) and W_q = w~ * beta:
+ *   dr = dy . W_q,  dW = dy^T . x_q,
+ *   dx = inv * gamma * dr - x * inv^3 * (sum_k gamma_k dr_k x_k) / K,
+ *   dgamma = sum over tokens of dr * x * inv,  inv = 1 / sqrt(sum x^2 / K + eps).
+ * dy: bf16 [M][N]; x, gamma, eps, packed, scale as for the forward;
+ * dx: bf16 [M][K]; dgamma: fp32 [K]; dW: fp32 [N][K] (the latent weights'
+ * gradient); all overwritten.  The two products are bf16 GEMMs with fp32
+ * accumulation (cuBLAS, opened on the first call; MMF_ERR_CUDA if it cannot
+ * be loaded); dy * absmax / 127 is rounded to bf16 for dW.  workspace: at
+ * least mmf_bwd_workspace_bytes(M, K, N) bytes, no initialisation needed.
+ * Sizes as the forward, with M * N and M * K below 2^31 and M <= 4194240.
+ */
+size_t mmf_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N);
+int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma,
+                      float eps, const uint32_t* packed, const float* scale,
+                      int64_t M, int64_t K, int64_t N, uint16_t* dx,
+                      float* dgamma, float* dW, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
 /* Flags of mmf_bitlinear_fwd_group. */
 #define MMF_FWD_PDL 1u   /* launch as a programmatic dependent of the kernel before it on the stream (see below) */
 #define MMF_MAX_GROUP 8  /* projections per mmf_bitlinear_fwd_group call */

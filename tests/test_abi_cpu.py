@@ -153,3 +153,13 @@ def test_mlgru_scan_argument_errors(L):
     assert f(A, None, A, None, 1, 4, 64, A, A, None) == 1   # missing input
     assert f(A, A, A, MIS, 1, 4, 64, A, A, None) == 3       # misaligned h0
     assert f(None, None, None, None, 0, 4, 64, None, None, None) == 0  # empty
+
+
+def test_bwd_argument_errors(L):
+    f = L.mmf_bitlinear_bwd
+    need = L.mmf_bwd_workspace_bytes(64, 256, 128)
+    assert need >= 64 * 256 * 4
+    assert f(A, A, A, 1e-6, A, A, 64, 256, 128, A, A, A, None, 0, None) == 1       # no workspace
+    assert f(A, A, A, 1e-6, A, A, 64, 100, 128, A, A, A, A, need, None) == 2       # bad K
+    assert f(A, A, A, 1e-6, A, A, 64, 256, 128, A, A, MIS, A, need, None) == 3     # misaligned dW
+    assert f(A, A, A, 1e-6, A, A, 64, 256, 128, A, A, A, A, need - 1, None) == 4   # short workspace

@@ -334,6 +334,28 @@ def test_mlgru_scan_continues_across_calls():
     assert ((both - o.float()).abs() <= o.float().abs() * 2.0 ** -7 + 1e-6).all()
 
 
+# -- backward with the straight-through estimator --------------------------------------------
+
+@pytest.mark.parametrize("M,K,N", [(1, 256, 128), (16, 512, 256), (64, 1024, 300), (300, 384, 1024),
+                                   (1000, 2048, 512)])
+def test_bwd_parity(oracle, M, K, N):
+    x, g, W = make_layer(24, M, K, N)
+    dy = I.activations(24, M, N, index=7)
+    packed, scale = _pack(W)
+    dx, dg, dW = mmf.bitlinear_bwd(dy.to(DEV), x.to(DEV), g.to(DEV), packed, scale, EPS)
+    torch.cuda.synchronize()
+    wt, beta = oracle.absmean_ternary(W.numpy(), EPS_W)
+    dx_ref, dg_ref, dW_ref = oracle.bitlinear_bwd(bits_np(dy), bits_np(x), g.numpy(), EPS, wt, beta)
+    # bf16 GEMM operands (dy * absmax / 127 rounded to bf16) and fp32 accumulation:
+    # errors well inside the layer's 1e-2 bar, relative to each output's scale
+    def rel(a, b):
+        b = np.asarray(b, dtype=np.float64)
+        return np.abs(np.asarray(a, dtype=np.float64) - b).max() / max(np.abs(b).max(), 1e-30)
+    assert rel(bf16_to_f64(bits_np(dx.cpu())), bf16_to_f64(dx_ref)) <= 1e-2
+    assert rel(dg.cpu().numpy(), dg_ref) <= 1e-3
+    assert rel(dW.cpu().numpy(), dW_ref) <= 1e-2
+
+
 def test_empty_problems():
     K, N = 256, 64
     x = torch.zeros(0, K, dtype=torch.bfloat16, device=DEV)
