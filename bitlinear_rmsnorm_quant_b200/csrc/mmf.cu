@@ -118,7 +118,8 @@ mmf_status device_state(DeviceState** out) {
         if (e == cudaSuccess) e = set_gemv_attrs<6>();
         if (e == cudaSuccess) e = set_gemv_attrs<7>();
         if (e == cudaSuccess) e = set_gemv_attrs<8>();
-        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_stream_kernel, quant_stream_smem(kMaxQuantStreamK));
+        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_stream_kernel<1>, quant_stream_smem(kMaxQuantStreamK, 1));
+        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_stream_kernel<2>, quant_stream_smem(kMaxQuantStreamK / 2, 2));
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8>, 2 * kMaxK);  // one row of the largest K
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8, true>, 2 * kMaxK);
         if (e != cudaSuccess) return MMF_ERR_CUDA;
@@ -278,17 +279,26 @@ mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_
     if (M < kQuantWarpRowMinM || K > kMaxQuantStreamK)  // one CTA of 8 warps per row
         return launch(rmsnorm_quant_kernel<8>, dim3(static_cast<unsigned>(M)), dim3(256), static_cast<size_t>(K) * 2,
                       s, pdl, x, gamma, eps, static_cast<int>(K), M, q, absmax, qsum, static_cast<const uint16_t*>(nullptr));
-    // persistent: as many CTAs as fit on the SMs at once, never more than the rows need
-    const size_t smem = quant_stream_smem(static_cast<int>(K));
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rmsnorm_quant_stream_kernel, kQuantStreamWarps * 32,
-                                                      smem) != cudaSuccess || per_sm < 1)
-        return MMF_ERR_CUDA;
-    int64_t grid = static_cast<int64_t>(per_sm) * num_sms;
+    // persistent: as many CTAs as fit on the SMs at once, never more than the
+    // rows need; two row buffers per warp unless that leaves one CTA per SM
+    int per_sm[2] = {0, 0};
+    for (int nb = 1; nb <= 2; ++nb) {
+        const size_t smem = quant_stream_smem(static_cast<int>(K), nb);
+        if (smem > quant_stream_smem(kMaxQuantStreamK, 1)) continue;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                &per_sm[nb - 1], nb == 1 ? rmsnorm_quant_stream_kernel<1> : rmsnorm_quant_stream_kernel<2>,
+                kQuantStreamWarps * 32, smem) != cudaSuccess)
+            return MMF_ERR_CUDA;
+    }
+    const int nb = per_sm[1] >= 2 ? 2 : 1;
+    if (per_sm[nb - 1] < 1) return MMF_ERR_CUDA;
+    int64_t grid = static_cast<int64_t>(per_sm[nb - 1]) * num_sms;
     const int64_t need = (M + kQuantStreamWarps - 1) / kQuantStreamWarps;
     if (grid > need) grid = need;
-    return launch(rmsnorm_quant_stream_kernel, dim3(static_cast<unsigned>(grid)), dim3(kQuantStreamWarps * 32), smem,
-                  s, pdl, x, gamma, eps, static_cast<int>(K), M, q, absmax, qsum);
+    const size_t smem = quant_stream_smem(static_cast<int>(K), nb);
+    return launch(nb == 1 ? rmsnorm_quant_stream_kernel<1> : rmsnorm_quant_stream_kernel<2>,
+                  dim3(static_cast<unsigned>(grid)), dim3(kQuantStreamWarps * 32), smem, s, pdl, x, gamma, eps,
+                  static_cast<int>(K), M, q, absmax, qsum);
 }
 
 // The fused forward of `count` projections that share x.  Arguments checked.

@@ -203,29 +203,34 @@ __global__ void __launch_bounds__(kQuantCtaWarps * 32) rmsnorm_quant_kernel(cons
 }
 
 // Large M: a persistent grid; warp w of the grid takes rows w, w + W, w + 2W,
-// ... (W warps in the grid) and double-buffers them, so the bulk copy of its
-// next row is in flight while it works on the current one.  Each row: the sum
-// of squares in fp64 (exact for bf16 squares, so the order of the additions
-// does not matter), the absmax of r = (x * inv) * gamma, then the codes.  A
-// code is rounded by one float addition: in [2^23, 2^24) consecutive floats
-// are 1 apart, so adding 1.5 * 2^23 to v = r * s (|v| <= 127 up to one ulp,
-// since s = 127 / a and a >= |r|) rounds v to the nearest integer, ties to
-// even, and leaves it in the low byte (1.5 * 2^23 has a zero low byte).  The
-// same integer as rint(v), which is already within [-127, 127], so the clamp
-// of the definition never changes a code.  Four bytes are packed with byte
-// permutes and summed with one DP4A.
+// ... (W warps in the grid).  With NB = 2 row buffers per warp the bulk copy
+// of its next row is in flight while it works on the current one; with NB = 1
+// the next row is requested when the current one is done, and the other warps
+// of the SM hide the wait (the launch takes NB = 1 when two buffers per warp
+// would leave fewer than two CTAs on an SM, as at K = 5632).  Each row: the
+// sum of squares in fp64 (exact for bf16 squares, so the order of the
+// additions does not matter), the absmax of r = (x * inv) * gamma, then the
+// codes.  A code is rounded by one float addition: in [2^23, 2^24)
+// consecutive floats are 1 apart, so adding 1.5 * 2^23 to v = r * s (|v| <=
+// 127 up to one ulp, since s = 127 / a and a >= |r|) rounds v to the nearest
+// integer, ties to even, and leaves it in the low byte (1.5 * 2^23 has a zero
+// low byte).  The same integer as rint(v), which is already within
+// [-127, 127], so the clamp of the definition never changes a code.  Four
+// bytes are packed with byte permutes and summed with one DP4A.
 constexpr int kQuantStreamWarps = 8;
-constexpr int kMaxQuantStreamK = 6400;  // gamma + 8 warps x 2 rows of bf16 within the 227 KB of one CTA
+constexpr int kMaxQuantStreamK = 11264;  // gamma + 8 warps x 1 row of bf16 within the 227 KB of one CTA
 
-__host__ __device__ inline size_t quant_stream_smem(int K) {
-    return static_cast<size_t>(4) * K + static_cast<size_t>(kQuantStreamWarps) * 2 * 2 * static_cast<size_t>(K);
+__host__ __device__ inline size_t quant_stream_smem(int K, int NB) {
+    return static_cast<size_t>(4) * K + static_cast<size_t>(kQuantStreamWarps) * NB * 2 * static_cast<size_t>(K);
 }
 
+template <int NB>
 __global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ gamma, float eps, int K, int64_t M,
     int8_t* __restrict__ q, float* __restrict__ absmax, int* __restrict__ qsum) {
-    extern __shared__ __align__(128) uint4 smem_q[];  // gamma fp32 [K], then [warp][2 buffers][K/8 chunks]
-    __shared__ __align__(8) uint64_t row_bar[kQuantStreamWarps][2];
+    static_assert(NB == 1 || NB == 2, "one or two row buffers per warp");
+    extern __shared__ __align__(128) uint4 smem_q[];  // gamma fp32 [K], then [warp][NB buffers][K/8 chunks]
+    __shared__ __align__(8) uint64_t row_bar[kQuantStreamWarps][NB];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int C = K >> 3;
     float4* gamma_s = reinterpret_cast<float4*>(smem_q);
@@ -233,10 +238,10 @@ __global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_k
     const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
     const int64_t gw = static_cast<int64_t>(blockIdx.x) * kQuantStreamWarps + warp;
     const int64_t TW = static_cast<int64_t>(gridDim.x) * kQuantStreamWarps;
-    auto buf = [&](int b) { return xs_all + (static_cast<size_t>(warp) * 2 + b) * C; };
+    auto buf = [&](int b) { return xs_all + (static_cast<size_t>(warp) * NB + b) * C; };
     if (lane == 0) {
-        mbar_init(&row_bar[warp][0], 1);
-        mbar_init(&row_bar[warp][1], 1);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) mbar_init(&row_bar[warp][b], 1);
         mbar_fence_init();
     }
     // gamma once per CTA into shared memory (read by every row, twice)
@@ -258,19 +263,21 @@ __global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_k
     const float4* g4 = gamma_s;
     int i = 0;
     for (int64_t m = gw; m < M; m += TW, ++i) {
-        const int b = i & 1;
+        const int b = NB == 2 ? (i & 1) : 0;
+        const uint32_t parity = static_cast<uint32_t>(NB == 2 ? (i >> 1) & 1 : i & 1);
         const bool next = m + TW < M;
-        if (next) issue(m + TW, b ^ 1);  // that buffer's last row was finished in the previous iteration
+        if (NB == 2 && next) issue(m + TW, b ^ 1);  // that buffer's last row was finished in the previous iteration
         int abort_flag = 0;
-        if (!__all_sync(0xffffffffu, mbar_wait(&row_bar[warp][b], (i >> 1) & 1, &abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&row_bar[warp][b], parity, &abort_flag))) {
             int no_abort = 0;  // let the copies in flight land in this CTA's shared memory
-            mbar_wait(&row_bar[warp][b], (i >> 1) & 1, &no_abort);
-            if (next) mbar_wait(&row_bar[warp][b ^ 1], ((i + 1) >> 1) & 1, &no_abort);
+            mbar_wait(&row_bar[warp][b], parity, &no_abort);
+            if (NB == 2 && next) mbar_wait(&row_bar[warp][b ^ 1], ((i + 1) >> 1) & 1, &no_abort);
             return;
         }
         const uint4* xs = buf(b);
 
         double s2[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 2
         for (int c = lane; c < C; c += 32) {
             float f[8];
             unpack_bf16x8(xs[c], f);
@@ -282,6 +289,7 @@ __global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_k
         const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
 
         float amax[2] = {0.0f, 0.0f};
+#pragma unroll 2
         for (int c = lane; c < C; c += 32) {
             float f[8];
             unpack_bf16x8(xs[c], f);
@@ -298,6 +306,7 @@ __global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_k
 
         int qs = 0;
         uint2* qr = reinterpret_cast<uint2*>(q + m * static_cast<int64_t>(K));
+#pragma unroll 2
         for (int c = lane; c < C; c += 32) {
             float f[8];
             unpack_bf16x8(xs[c], f);
@@ -319,6 +328,7 @@ __global__ void __launch_bounds__(kQuantStreamWarps * 32) rmsnorm_quant_stream_k
             if (qsum) qsum[m] = qs;
         }
         __syncwarp();  // every lane is done with this buffer before it is refilled
+        if (NB == 1 && next) issue(m + TW, 0);
     }
 }
 

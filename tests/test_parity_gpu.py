@@ -82,9 +82,11 @@ def test_pack_special_matrices(oracle):
 
 @pytest.mark.parametrize("M,K,outliers", [(16, 256, 0.0), (5, 128, 0.0), (300, 2048, 0.0), (37, 6912, 0.01),
                                           (64, 5632, 0.0),
-                                          # large M: the persistent double-buffered quantiser
+                                          # large M: the persistent streaming quantiser
                                           (4100, 1024, 0.0), (4096, 7168, 0.01), (5000, 128, 0.0),
-                                          (4097, 7296, 0.0)])
+                                          (4097, 7296, 0.0),
+                                          # one row buffer per warp up to its largest K; beyond it, a CTA per row
+                                          (4096, 11264, 0.0), (4096, 11392, 0.01)])
 def test_quantize_act(oracle, M, K, outliers):
     x, g, _ = make_layer(9, M, K, 1, outlier_frac=outliers)
     q, a = mmf.quantize_act(x.to(DEV), g.to(DEV), EPS)
