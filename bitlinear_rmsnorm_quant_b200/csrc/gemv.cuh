@@ -149,7 +149,6 @@ __global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_k
     __shared__ __align__(8) uint64_t full_bar[kGemvMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kGemvMaxStages];
     __shared__ __align__(8) uint64_t act_bar;
-    __shared__ int qsum_s[MT];
     __shared__ float deq_s[MT];
     __shared__ float beta_s[kGemvMaxProj];
     __shared__ double red_d[NW];
@@ -258,7 +257,7 @@ __global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_k
     const bool act_ok = mbar_wait(&act_bar, 0, &abort_flag);
     if constexpr (FUSED) {
         const int C8 = K >> 3;
-        const uint4* xr = reinterpret_cast<const uint4*>(x_s + static_cast<size_t>(m) * K);
+        uint4* xr = reinterpret_cast<uint4*>(x_s + static_cast<size_t>(m) * K);
         const float4* g4 = reinterpret_cast<const float4*>(gamma_s);
         double s2 = 0.0;
         if (active && act_ok) {
@@ -267,14 +266,16 @@ __global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_k
                 if constexpr (GLU) {
                     // the GLU gated product replaces x (this thread alone reads chunk c later)
                     v = glu_gate8(v, __ldg(reinterpret_cast<const uint4*>(p.u + static_cast<size_t>(m) * K) + c));
-                    const_cast<uint4*>(xr)[c] = v;
+                    xr[c] = v;
                 }
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                double sq[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const double lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
-                    s2 += lo * lo + hi * hi;
+                    sq[i] = lo * lo + hi * hi;
                 }
+                s2 += (sq[0] + sq[1]) + (sq[2] + sq[3]);  // exact sums: the order does not matter
             }
         }
         s2 = warp_sum_f64(s2);
@@ -305,7 +306,11 @@ __global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_k
         amax = tree_max<WPT>(red_f + w0);
         const float a = fmaxf(amax, 1e-5f);
         const float s = __fdiv_rn(127.0f, a);
+        if (active && tg == 0) deq_s[m] = __fdiv_rn(a, 127.0f);  // published by the barrier below
 
+        // codes: v = r * s (|v| <= 127 up to an ulp, as a >= |r|) is rounded to
+        // the nearest integer, ties to even, by adding 1.5 * 2^23, which leaves
+        // the code in the low byte; the clamp of the definition never acts
         int qs = 0;
         if (active && act_ok) {
             int8_t* qrow = q_s + static_cast<size_t>(m) * K;
@@ -315,27 +320,24 @@ __global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_k
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
                 const float4 ga = g4[2 * c], gb = g4[2 * c + 1];
                 const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-                uint32_t out[2] = {0u, 0u};
+                uint32_t cb[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float xv =
                         (i & 1) ? __uint_as_float(w[i >> 1] & 0xFFFF0000u) : __uint_as_float(w[i >> 1] << 16);
-                    const int code = quant_code(__fmul_rn(__fmul_rn(xv, inv), g[i]), s);
-                    qs += code;
-                    out[i >> 2] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (i & 3));
+                    cb[i] = __float_as_uint(__fadd_rn(__fmul_rn(__fmul_rn(__fmul_rn(xv, inv), g[i]), s), 12582912.0f));
                 }
+                const uint32_t o0 = __byte_perm(__byte_perm(cb[0], cb[1], 0x0040), __byte_perm(cb[2], cb[3], 0x0040), 0x5410);
+                const uint32_t o1 = __byte_perm(__byte_perm(cb[4], cb[5], 0x0040), __byte_perm(cb[6], cb[7], 0x0040), 0x5410);
+                qs = __dp4a(static_cast<int>(o0), 0x01010101, qs);
+                qs = __dp4a(static_cast<int>(o1), 0x01010101, qs);
                 // codes k = 8c .. 8c+7 -> unit (c/8, (c%8)/2), half c%2 of the t-major layout
                 *reinterpret_cast<uint2*>(qrow + 16 * (((c & 7) >> 1) * C64 + (c >> 3)) + 8 * (c & 1)) =
-                    make_uint2(out[0], out[1]);
+                    make_uint2(o0, o1);
             }
         }
         qs = __reduce_add_sync(0xffffffffu, qs);
         if (lane == 0) red_i[warp] = qs;
-        gemv_compute_sync<NW>();
-        if (active && tg == 0) {
-            qsum_s[m] = tree_sum<WPT>(red_i + w0);
-            deq_s[m] = __fdiv_rn(a, 127.0f);
-        }
     } else {
         int qs = 0;
         if (active && act_ok) {
@@ -356,22 +358,47 @@ __global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_k
         }
         qs = __reduce_add_sync(0xffffffffu, qs);
         if (lane == 0) red_i[warp] = qs;
-        gemv_compute_sync<NW>();
-        if (active && tg == 0) {
-            qsum_s[m] = tree_sum<WPT>(red_i + w0);
-        }
     }
-    gemv_compute_sync<NW>();
-    if (!act_ok) return;
+    // codes, per-warp code sums and dequantisation factors visible; the warps
+    // agree on whether gamma arrived
+    if (!named_barrier_and<1, NW * 32>(act_ok)) return;
+    // the sum of the codes of each token, from its warps' partial sums in index order
+    int qsum_r[MT];
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm) qsum_r[mm] = tree_sum<WPT>(red_i + mm * WPT);
 
     // ---------------- contraction over the staged rows
-    // Blocks of 8 rows go round-robin to the compute warps over the whole slab.
+    // Blocks of 8 rows go round-robin to the compute warps over the whole slab
+    // (for one token and a resident slab, possibly items of 4 rows instead).
     const int rsub = lane >> 3;    // lane handles rows rsub and rsub + 4 of a block
     const int l8 = lane & 7;       // lane within the row
     const int C = K >> 6;          // 16-byte chunks (64 weights) per row
     const int bps = p.rows_per_stage / kGemvBlockRows;
     const int nblocks = (nrows + kGemvBlockRows - 1) / kGemvBlockRows;
 
+    auto finish_row = [&](const int (&ac)[MT][4], int s, int rl, bool valid) {
+        const int r = row0 + s * p.rows_per_stage + rl;
+        const int g = gemv_proj_of(p, valid ? r : row0);
+        const int n = r - p.row_start[g];
+        const int Ng = p.row_start[g + 1] - p.row_start[g];
+#pragma unroll
+        for (int mm = 0; mm < MT; ++mm) {
+            int t = ac[mm][0] + (ac[mm][1] >> 2) + (ac[mm][2] >> 4) + (ac[mm][3] >> 6);
+            t += __shfl_xor_sync(0xffffffffu, t, 1);
+            t += __shfl_xor_sync(0xffffffffu, t, 2);
+            t += __shfl_xor_sync(0xffffffffu, t, 4);
+            if (valid && l8 == 0 && mm < p.M) {
+                const int v = t - qsum_r[mm];
+                if constexpr (FUSED) {
+                    const float cm = __fmul_rn(deq_s[mm], beta_s[g]);
+                    const __nv_bfloat16 yb = __float2bfloat16_rn(__fmul_rn(static_cast<float>(v), cm));
+                    p.y[g][static_cast<size_t>(mm) * Ng + n] = __bfloat16_as_ushort(yb);
+                } else {
+                    p.acc[static_cast<size_t>(mm) * Ng + n] = v;
+                }
+            }
+        }
+    };
     auto do_block = [&](int gb, int s, int slot) {
         const int rs = min(p.rows_per_stage, nrows - s * p.rows_per_stage);
         const int b = gb - s * bps;
@@ -446,40 +473,64 @@ __global__ void __launch_bounds__(gemv_threads(MT), gemv_ctas_per_sm(MT)) gemv_k
             }
         }
         }
-        auto finish_row = [&](const int (&ac)[MT][4], int rl, bool valid) {
-            const int r = row0 + s * p.rows_per_stage + rl;
-            const int g = gemv_proj_of(p, valid ? r : row0);
-            const int n = r - p.row_start[g];
-            const int Ng = p.row_start[g + 1] - p.row_start[g];
+        finish_row(acc0, s, rl0, v0);
+        finish_row(acc1, s, rl1, v1);
+    };
+
+    // One token, whole slab resident: items of 4 rows (lane group rsub takes
+    // row rsub), so a slab of few rows spreads over more warps.
+    auto do_rows4 = [&](int it) {
+        const int s = (4 * it) / p.rows_per_stage;
+        const int rs = min(p.rows_per_stage, nrows - s * p.rows_per_stage);
+        const int rl = 4 * it - s * p.rows_per_stage + rsub;
+        const bool v = rl < rs;
+        const uint4* wp = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(s) * p.stage_bytes +
+                                                         static_cast<size_t>(v ? rl : 0) * rowbytes);
+        int a[4][4];
 #pragma unroll
-            for (int mm = 0; mm < MT; ++mm) {
-                int t = ac[mm][0] + (ac[mm][1] >> 2) + (ac[mm][2] >> 4) + (ac[mm][3] >> 6);
-                t += __shfl_xor_sync(0xffffffffu, t, 1);
-                t += __shfl_xor_sync(0xffffffffu, t, 2);
-                t += __shfl_xor_sync(0xffffffffu, t, 4);
-                if (valid && l8 == 0 && mm < p.M) {
-                    const int v = t - qsum_s[mm];
-                    if constexpr (FUSED) {
-                        const float cm = __fmul_rn(deq_s[mm], beta_s[g]);
-                        const __nv_bfloat16 yb = __float2bfloat16_rn(__fmul_rn(static_cast<float>(v), cm));
-                        p.y[g][static_cast<size_t>(mm) * Ng + n] = __bfloat16_as_ushort(yb);
-                    } else {
-                        p.acc[static_cast<size_t>(mm) * Ng + n] = v;
-                    }
-                }
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) a[t][j] = 0;
+#pragma unroll 2
+        for (int c = l8; c < C; c += 8) {
+            const uint4 wa = wp[c];
+            const uint32_t da[4] = {wa.x, wa.y, wa.z, wa.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const uint4 qv = *reinterpret_cast<const uint4*>(q_s + 16 * (t * C + c));
+                a[t][0] = dp4a_us(da[t] & 0x03030303u, qv.x, a[t][0]);
+                a[t][1] = dp4a_us(da[t] & 0x0C0C0C0Cu, qv.y, a[t][1]);
+                a[t][2] = dp4a_us(da[t] & 0x30303030u, qv.z, a[t][2]);
+                a[t][3] = dp4a_us(da[t] & 0xC0C0C0C0u, qv.w, a[t][3]);
             }
-        };
-        finish_row(acc0, rl0, v0);
-        finish_row(acc1, rl1, v1);
+        }
+        int acc[MT][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[0][j] = (a[0][j] + a[1][j]) + (a[2][j] + a[3][j]);
+        finish_row(acc, s, rl, v);
     };
 
     if (nst <= S) {
         // The ring holds the whole slab: every slot is filled once (phase 0),
         // so a warp waits only for the stage of each of its blocks.
-        for (int gb = warp; gb < nblocks; gb += NW) {
-            const int s = gb / bps;
-            if (!mbar_wait(&full_bar[s], 0, &abort_flag)) break;
-            do_block(gb, s, s);
+        // one token: 4-row items when 8-row blocks would leave warps idle and the
+        // busiest warp gets fewer rows
+        const int n4 = (nrows + 3) / 4;
+        bool rows4 = false;
+        if constexpr (MT == 1) rows4 = nblocks < NW && (n4 + NW - 1) / NW * 4 < kGemvBlockRows;
+        if (rows4) {
+            if constexpr (MT == 1) {
+                for (int it = warp; it < n4; it += NW) {
+                    if (!mbar_wait(&full_bar[(4 * it) / p.rows_per_stage], 0, &abort_flag)) break;
+                    do_rows4(it);
+                }
+            }
+        } else {
+            for (int gb = warp; gb < nblocks; gb += NW) {
+                const int s = gb / bps;
+                if (!mbar_wait(&full_bar[s], 0, &abort_flag)) break;
+                do_block(gb, s, s);
+            }
         }
     } else {
         // Slots are refilled: every warp walks the stages in order and releases
