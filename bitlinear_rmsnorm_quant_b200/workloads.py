@@ -95,6 +95,13 @@ PREFILL_1P3B = Workload(
     projections=(Projection("proj", 2048, 2048, 0), Projection("up", 2048, 5632, 1),
                  Projection("down", 5632, 2048, 2)))
 
+PREFILL_2P7B = Workload(
+    "prefill-2.7b", "prefill at 2.7B width, M=8192: 2560->2560, 2560->6912, 6912->2560; 1% outlier channels x20",
+    seed=6, M=8192,
+    projections=(Projection("proj", 2560, 2560, 0), Projection("up", 2560, 6912, 1),
+                 Projection("down", 6912, 2560, 2)),
+    outlier_frac=0.01)
+
 TRAIN_FWD_1P3B = Workload(
     "train-fwd-1.3b",
     "training-batch forward at 1.3B width, M=2^8*2048=524288, full BitLinear set "
@@ -103,4 +110,4 @@ TRAIN_FWD_1P3B = Workload(
 
 
 ALL = {w.name: w for w in (SMOKE, DECODE_370M, decode_2p7b(1), decode_2p7b(8),
-                           decode_2p7b(32), PREFILL_1P3B, TRAIN_FWD_1P3B)}
+                           decode_2p7b(32), PREFILL_1P3B, PREFILL_2P7B, TRAIN_FWD_1P3B)}

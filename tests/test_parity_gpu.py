@@ -194,12 +194,12 @@ def test_decode_configs(oracle, wl):
         _layer_parity(oracle, x, g, W)
 
 
-def test_prefill_config_sampled(oracle):
+@pytest.mark.parametrize("wl", [WL.PREFILL_1P3B, WL.PREFILL_2P7B], ids=lambda w: w.name)
+def test_prefill_config_sampled(oracle, wl):
     """Full prefill size (M=8192) on the GPU; the oracle checks 48 sampled tokens."""
-    wl = WL.PREFILL_1P3B
     rng = np.random.default_rng(5)
     for p in wl.projections:
-        x, g, W = make_layer(wl.seed, wl.M, p.K, p.N, index=p.input_index)
+        x, g, W = make_layer(wl.seed, wl.M, p.K, p.N, index=p.input_index, outlier_frac=wl.outlier_frac)
         tokens = np.sort(rng.choice(wl.M, 48, replace=False))
         _layer_parity(oracle, x, g, W, sample_tokens=tokens)
 
