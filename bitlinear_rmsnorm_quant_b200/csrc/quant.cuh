@@ -45,9 +45,6 @@ struct AddOp {
     template <typename T>
     __device__ __forceinline__ T operator()(T a, T b) const { return a + b; }
 };
-struct MaxOp {
-    __device__ __forceinline__ float operator()(float a, float b) const { return fmaxf(a, b); }
-};
 
 // 8 bf16 in a uint4 -> 8 floats
 __device__ __forceinline__ void unpack_bf16x8(const uint4& v, float (&f)[8]) {
