@@ -118,8 +118,9 @@ mmf_status device_state(DeviceState** out) {
         if (e == cudaSuccess) e = set_gemv_attrs<6>();
         if (e == cudaSuccess) e = set_gemv_attrs<7>();
         if (e == cudaSuccess) e = set_gemv_attrs<8>();
+        // both buffer counts may be asked about up to the streaming kernel's limit
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_stream_kernel<1>, quant_stream_smem(kMaxQuantStreamK, 1));
-        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_stream_kernel<2>, quant_stream_smem(kMaxQuantStreamK / 2, 2));
+        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_stream_kernel<2>, quant_stream_smem(kMaxQuantStreamK, 1));
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8>, 2 * kMaxK);  // one row of the largest K
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8, true>, 2 * kMaxK);
         if (e != cudaSuccess) return MMF_ERR_CUDA;
