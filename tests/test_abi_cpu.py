@@ -163,3 +163,37 @@ def test_bwd_argument_errors(L):
     assert f(A, A, A, 1e-6, A, A, 64, 100, 128, A, A, A, A, need, None) == 2       # bad K
     assert f(A, A, A, 1e-6, A, A, 64, 256, 128, A, A, MIS, A, need, None) == 3     # misaligned dW
     assert f(A, A, A, 1e-6, A, A, 64, 256, 128, A, A, A, A, need - 1, None) == 4   # short workspace
+
+
+def test_shape_limits(L):
+    f = L.mmf_bitlinear_fwd
+    big_ws = 1 << 62  # claimed workspace size: the shape checks come first
+    # tokens beyond the grid's token-tile limit; a weight matrix beyond 2^40 elements
+    assert f(A, A, 1e-6, A, A, 65535 * 256 + 1, 128, 16, A, A, big_ws, None) == 2
+    assert f(A, A, 1e-6, A, A, 16, 65536, (1 << 24) + 16, A, A, big_ws, None) == 2
+    # the allocation-free call refuses shapes whose workspace exceeds its static scratch
+    assert L.mmf_bitlinear_fwd_noalloc(A, A, 1e-6, A, A, 65536, 2048, 2048, A, None) == 4
+    # the backward's dgamma grid limit
+    need = L.mmf_bwd_workspace_bytes(65535 * 64 + 1, 128, 16)
+    assert L.mmf_bitlinear_bwd(A, A, A, 1e-6, A, A, 65535 * 64 + 1, 128, 16, A, A, A, A, need, None) == 2
+    # the timeout self-test needs a limit within the library's own
+    assert L.mmf_selftest_timeout(0, None, None) == 1
+
+
+def test_workspace_sizes_follow_the_path(L):
+    # the decode path (up to 8 tokens whose activations fit in shared memory) needs none;
+    # the large-M path needs the codes, the per-token absmax and code sums
+    for K in (128, 2560, 6912):
+        assert L.mmf_workspace_bytes(1, K, 256) == 0
+        assert L.mmf_workspace_bytes(8, K, 256) == 0
+        assert L.mmf_workspace_bytes(9, K, 256) >= 9 * K + 8 * 9
+        assert L.mmf_workspace_bytes(8192, K, 256) >= 8192 * K + 8 * 8192
+    # a single token too wide for the decode kernel's shared memory takes the large-M path
+    assert L.mmf_workspace_bytes(1, 65536, 256) >= 65536
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device path")
+def test_largest_k_passes_the_shape_checks(L):
+    # K = 65536 is inside the limit: the call gets as far as looking for a device
+    assert L.mmf_bitlinear_fwd(A, A, 1e-6, A, A, 1, 65536, 16, A, A, 1 << 30, None) == 7
+    assert L.mmf_quantize_act(A, A, 1e-6, 4096, 65536, A, A, None) == 7
