@@ -2,19 +2,25 @@
 """Benchmark of the fused RMSNorm + BitLinear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--layers L]
+                    [--workload NAME] [--layers L] [--secondary LIST]
 
-Prints ONE JSON line (rank 0).  Default workload: decode at the 2.7B width,
-M = 1 token, the 7-projection BitLinear set (4x 2560->2560, 2x 2560->6912,
-6912->2560), repeated over L = 32 layer sets with distinct weights so the
-packed weights (634 MB) exceed L2 and stream from HBM every step.
+Prints ONE JSON line (rank 0).  Default workload: the training-batch forward
+at the 1.3B width, M = 2^8 x 2048 = 524288 tokens through the full BitLinear
+set of one layer (4x 2048->2048, 2x 2048->5632, 5632->2048), each projection
+group with its own fused RMSNorm + int8 quantisation: the largest
+configuration that fits one GPU.  The same line carries a `secondary` list
+with the prefill step at the 2.7B width (the int8 tensor-core target) and the
+decode steps at the 2.7B width for 1, 8 and 32 tokens (the HBM target), each
+timed in the same run with its own step time, roofline, end-to-end figure and
+clock record.
 
 A step = one pass of the whole hot path (RMSNorm, int8 quantisation, ternary
 contraction, rescale: every projection of every layer set) over one batch of M
 tokens, replayed as one CUDA graph.  `value` = tokens/s through one layer set
-(M * L * n_gpus / step time), i.e. the decode rate of one token through the
-BitLinear set of one layer.  Weights are packed once, before timing (offline
-on the pages' terms).
+(M * L * n_gpus / step time).  Weights are packed once, before timing (offline
+on the pages' terms).  Decode steps repeat the layer set over L = 32 layer
+sets with distinct weights so that the packed weights (634 MB) exceed L2 and
+stream from HBM every step.
 
 --impl reference times the CPU oracle (the only reference this method has on
 the box), on bounded samples of the same workload.  Multi-GPU: one process per
@@ -43,14 +49,6 @@ from bitlinear_rmsnorm_quant_b200 import workloads as WL  # noqa: E402
 
 METRIC = "fused RMSNorm+BitLinear tokens/s; GB/s or int8 TOPS as % of B200 roofline"
 
-# DRAM bytes (read + write) per launch of the dominant kernel, mean over the
-# launch shapes of one layer set, from the ncu captures summarised in
-# profiles/.  An entry must be removed whenever its kernel changes.
-NCU_TRAFFIC = {
-    "decode-2.7b-m1": {"bytes_per_launch": 5029248, "source": "profiles/gemv_decode-2.7b-m1.md"},
-    "prefill-1.3b": {"bytes_per_launch": 40680000, "source": "profiles/gemm_tc_prefill-1.3b.md"},
-    "prefill-2.7b": {"bytes_per_launch": 58282325, "source": "profiles/gemm_tc_prefill-2.7b.md"},
-}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 2.0   # nominal dense ratio int8 : bf16 (4.5 : 2.25 POPS)
@@ -148,8 +146,10 @@ def run_scan(args, dist):
 
 def run_bwd(args, dist):
     """Backward of the three prefill projections at the 1.3B width (M = 8192):
-    two bf16 GEMMs each (dr and dW) plus the straight-through operand
-    preparation and the RMSNorm backward."""
+    per projection the quantiser (the forward's codes), the two tensor-core
+    products (dr = dy . w~ with the weights unpacked from their 2-bit codes,
+    dW = dy^T . x_q with the codes scaled on the way in), the RMSNorm backward
+    and the two-stage dgamma sum: 6 launches, all this library's kernels."""
     from bitlinear_rmsnorm_quant_b200 import mmf
     wl = WL.PREFILL_1P3B
     M = wl.M
@@ -207,9 +207,10 @@ def run_bwd(args, dist):
         "config": {"workload": "bwd-prefill-1.3b", "M": M, "projections": [f"{p.K}->{p.N}" for p in wl.projections],
                    "parallelism": f"dp{dist.world} (replicas)"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None, "kernel": "cuBLAS bf16 GEMMs + own kernels",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "gemm_bwd_kernel (tcgen05 kind::f16), whole backward step",
                      "peak_source": f"{peak_src} bf16_tflops", "algorithmic_flops_per_step": flops},
-        "gpu_launches": 7 * len(items) * args.steps,   # ours; cuBLAS adds its own GEMM kernels
+        "gpu_launches": 6 * len(items) * args.steps,
         "clocks": clocks.summary(),
     }
 
@@ -372,7 +373,10 @@ WORKLOADS = {
     "bwd-prefill-1.3b": (None, 1),  # straight-through backward of the prefill projections (run_bwd)
 }
 SCAN_SHAPE = (4, 2048, 2048)        # sequences, tokens, channels: 4 x 2048 tokens at the 1.3B width
-DEFAULT_WORKLOAD = "decode-2.7b-m1"
+DEFAULT_WORKLOAD = "train-fwd-1.3b"
+DEFAULT_SECONDARY = "prefill-2.7b,decode-2.7b-m1,decode-2.7b-m8,decode-2.7b-m32"
+E2E_SINGLE_SHOT_BYTES = 8 << 30     # above this x + y, the end-to-end step streams token chunks
+E2E_CHUNKS = 8
 
 
 def proj_bytes(M, K, N):
@@ -384,170 +388,294 @@ def proj_ops(M, K, N):
     return 2 * M * N * K
 
 
+def hbm_bound(wl) -> bool:
+    """Decode batches (M <= 32) are bound by streaming the packed weights: 2M
+    int8 operations per 0.25 byte is below the int8 ridge point of the chip."""
+    return wl.M <= 32
+
+
+# ----------------------------------------------------------------------------- copy kernel
+
+def time_hbm_copy(dev, nbytes: int = 1 << 30, reps: int = 10):
+    """The library's 128-bit streaming copy (mmf_hbm_copy) on 1 GiB: read +
+    write bytes per second, median of `reps` CUDA-event timings.  Stated next
+    to the measured copy bandwidth the HBM fractions use."""
+    from bitlinear_rmsnorm_quant_b200 import mmf
+    src = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    src.fill_(1)
+    for _ in range(3):
+        mmf.hbm_copy(src, dst)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mmf.hbm_copy(src, dst)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    mmf.check_async()
+    ms = statistics.median(times)
+    del src, dst
+    return {"kernel": "hbm_copy_kernel (mmf_hbm_copy)", "bytes_copied": nbytes,
+            "gbs": round(2 * nbytes / (ms / 1e3) / 1e9, 1), "ms": round(ms, 4),
+            "note": "read + write bytes / time, median of %d copies of 1 GiB" % reps}
+
+
 # ----------------------------------------------------------------------------- our arm
 
-def run_ours(args, dist: Dist):
-    from bitlinear_rmsnorm_quant_b200 import mmf
-    dev = torch.device("cuda", dist.local_rank)
-    torch.cuda.set_device(dev)
-    wl, default_layers = WORKLOADS[args.workload]
-    wl = wl()
-    L = args.layers or default_layers
-    M = wl.M
-    seed = wl.seed + 7919 * dist.rank  # each rank draws its own tokens and weights
+class Step:
+    """One workload's step: packed weights, inputs and outputs resident on the
+    device, the library calls of one step, and their CUDA graph."""
 
-    # -- weights: drawn on the device, packed once (offline), fp32 freed
-    packed, scales = {}, {}
-    for l in range(L):
+    def __init__(self, wl, L, dist, args):
+        from bitlinear_rmsnorm_quant_b200 import mmf
+        self.mmf = mmf
+        self.wl, self.L = wl, L
+        dev = torch.device("cuda", dist.local_rank)
+        self.dev = dev
+        M = wl.M
+        seed = wl.seed + 7919 * dist.rank  # each rank draws its own tokens and weights
+        # -- weights: drawn on the device, packed once (offline), fp32 freed
+        self.packed, self.scales = {}, {}
+        for l in range(L):
+            for j, p in enumerate(wl.projections):
+                W = I.latent_weights(seed, p.N, p.K, index=64 * l + j, device=dev)
+                self.packed[l, j], self.scales[l, j] = mmf.pack_ternary(W, wl.eps_w)
+                del W
+
+        # -- activations and outputs: views into one flat device buffer each
+        def carve(shapes):
+            offs, total = [], 0
+            for shp in shapes:
+                offs.append(total)
+                total += (math.prod(shp) + 7) // 8 * 8      # 16-byte aligned views
+            flat = torch.empty(max(total, 8), dtype=torch.bfloat16, device=dev)
+            return flat, [flat[o:o + math.prod(shp)].view(*shp) for o, shp in zip(offs, shapes)]
+
+        x_keys = [(l, idx) for l in range(L) for idx, _ in wl.inputs()]
+        self.x_flat, x_views = carve([(M, dict(wl.inputs())[idx]) for _, idx in x_keys])
+        self.xs = dict(zip(x_keys, x_views))
+        for (l, idx), xv in self.xs.items():
+            xv.copy_(I.activations(seed, M, xv.shape[1], index=64 * l + idx, outlier_frac=wl.outlier_frac,
+                                   device=dev))
+        self.gs = {(l, idx): I.gamma(seed, K, index=64 * l + idx, device=dev)
+                   for l in range(L) for idx, K in wl.inputs()}
+        y_keys = [(l, j) for l in range(L) for j in range(len(wl.projections))]
+        self.y_flat, y_views = carve([(M, wl.projections[j].N) for _, j in y_keys])
+        self.ys = dict(zip(y_keys, y_views))
+        self.groups = {}
         for j, p in enumerate(wl.projections):
-            W = I.latent_weights(seed, p.N, p.K, index=64 * l + j, device=dev)
-            packed[l, j], scales[l, j] = mmf.pack_ternary(W, wl.eps_w)
-            del W
-    # -- activations and outputs: views into one flat device buffer each, so the
-    #    end-to-end step is one H2D copy, the graph, and one D2H copy
-    def carve(shapes):
-        offs, total = [], 0
-        for shp in shapes:
-            offs.append(total)
-            total += (math.prod(shp) + 7) // 8 * 8      # 16-byte aligned views
-        flat = torch.empty(max(total, 8), dtype=torch.bfloat16, device=dev)
-        return flat, [flat[o:o + math.prod(shp)].view(*shp) for o, shp in zip(offs, shapes)]
+            self.groups.setdefault(p.input_index, []).append(j)
+        ws_need = max(max(mmf.workspace_bytes(M, wl.projections[js[0]].K,
+                                              sum(wl.projections[j].N for j in js)),
+                          max(mmf.workspace_bytes(M, wl.projections[j].K, wl.projections[j].N) for j in js))
+                      for js in self.groups.values())
+        self.ws = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=dev)
+        self.lib = mmf.lib()
+        self.flags = 0 if args.no_pdl else mmf.FWD_PDL
+        self.api, self.glu = args.api, args.glu
+        self.keep = []           # ctypes arrays that must outlive the graph
+        self.launches_per_step = 0
+        self.bytes_per_step = 0
+        self.ops_per_step = 0
+        self.calls = self.make_calls(0, M, count=True)
+        self.graph = None
 
-    x_keys = [(l, idx) for l in range(L) for idx, _ in wl.inputs()]
-    x_flat, x_views = carve([(M, dict(wl.inputs())[idx]) for _, idx in x_keys])
-    xs = dict(zip(x_keys, x_views))
-    for (l, idx), xv in xs.items():
-        xv.copy_(I.activations(seed, M, xv.shape[1], index=64 * l + idx, outlier_frac=wl.outlier_frac, device=dev))
-    gs = {(l, idx): I.gamma(seed, K, index=64 * l + idx, device=dev) for l in range(L) for idx, K in wl.inputs()}
-    y_keys = [(l, j) for l in range(L) for j in range(len(wl.projections))]
-    y_flat, y_views = carve([(M, wl.projections[j].N) for _, j in y_keys])
-    ys = dict(zip(y_keys, y_views))
-    by_input = {}
-    for p in wl.projections:
-        by_input.setdefault(p.input_index, []).append(p)
-    ws_need = max(max(mmf.workspace_bytes(M, ps[0].K, sum(p.N for p in ps)),  # one grouped call
-                      max(mmf.workspace_bytes(M, p.K, p.N) for p in ps))      # or single calls
-                  for ps in by_input.values())
-    ws = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=dev)
-    lib = mmf.lib()
-
-    # one call per (layer set, shared input): the token mixer's 4 projections,
-    # the channel mixer's gate/up pair and the down projection each share x
-    flags = 0 if args.no_pdl else mmf.FWD_PDL
-    calls = []          # (function, args without the stream)
-    keep = []           # ctypes arrays that must outlive the graph
-    launches_per_step = 0
-    bytes_per_step = 0
-    ops_per_step = 0
-    for l in range(L):
-        groups = {}
-        for j, p in enumerate(wl.projections):
-            groups.setdefault(p.input_index, []).append(j)
-        for idx, js in sorted(groups.items()):
-            K = wl.projections[js[0]].K
-            x, g = xs[l, idx], gs[l, idx]
-            names = [wl.projections[j].name for j in js]
-            if args.glu and names == ["down"]:
-                # the channel mixer's down projection reads this layer set's gate and up
-                # outputs through the fused GLU call (SiLU(g) * u formed while normalising)
-                jg = [j for j, p in enumerate(wl.projections) if p.name == "gate"][0]
-                ju = [j for j, p in enumerate(wl.projections) if p.name == "up"][0]
-                j = js[0]
-                p = wl.projections[j]
-                calls.append((lib.mmf_bitlinear_fwd_glu, (ys[l, jg].data_ptr(), ys[l, ju].data_ptr(), g.data_ptr(),
-                                                          wl.eps, packed[l, j].data_ptr(), scales[l, j].data_ptr(),
-                                                          M, p.K, p.N, ys[l, j].data_ptr(), ws.data_ptr(), ws.numel(),
-                                                          flags)))
-                launches_per_step += 1 if mmf.workspace_bytes(M, p.K, p.N) == 0 else 2
-                bytes_per_step += p.N * p.K // 4 + 2 * M * p.N + 4 + 2 * (2 * M * K) + 4 * K  # g and u, gamma
-                ops_per_step += proj_ops(M, p.K, p.N)
-                continue
-            if args.api == "group":
-                arr = mmf.projection_array([(packed[l, j], scales[l, j], ys[l, j], wl.projections[j].N) for j in js])
-                keep.append(arr)
-                calls.append((lib.mmf_bitlinear_fwd_group, (x.data_ptr(), g.data_ptr(), wl.eps, M, K, arr, len(js),
-                                                            ws.data_ptr(), ws.numel(), flags)))
-                tc = mmf.workspace_bytes(M, K, 1) > 0
-                launches_per_step += (1 + len(js)) if tc else 1
-            else:
-                for j in js:
+    def make_calls(self, t0, t1, count=False):
+        """The library calls of one step over tokens [t0, t1) (all of them for
+        the graph; a token chunk for the streamed end-to-end step)."""
+        wl, mmf, lib = self.wl, self.mmf, self.lib
+        Mc = t1 - t0
+        calls = []
+        for l in range(self.L):
+            for idx, js in sorted(self.groups.items()):
+                K = wl.projections[js[0]].K
+                x, g = self.xs[l, idx][t0:t1], self.gs[l, idx]
+                y = {j: self.ys[l, j][t0:t1] for j in range(len(wl.projections))}
+                names = [wl.projections[j].name for j in js]
+                if self.glu and names == ["down"]:
+                    # the channel mixer's down projection reads this layer set's gate and up
+                    # outputs through the fused GLU call (SiLU(g) * u formed while normalising)
+                    jg = [j for j, p in enumerate(wl.projections) if p.name == "gate"][0]
+                    ju = [j for j, p in enumerate(wl.projections) if p.name == "up"][0]
+                    j = js[0]
                     p = wl.projections[j]
-                    calls.append((lib.mmf_bitlinear_fwd, (x.data_ptr(), g.data_ptr(), wl.eps, packed[l, j].data_ptr(),
-                                                          scales[l, j].data_ptr(), M, p.K, p.N, ys[l, j].data_ptr(),
-                                                          ws.data_ptr(), ws.numel())))
-                    launches_per_step += 1 if mmf.workspace_bytes(M, p.K, p.N) == 0 else 2
-            for j in js:
-                p = wl.projections[j]
-                bytes_per_step += p.N * p.K // 4 + 2 * M * p.N + 4
-                ops_per_step += proj_ops(M, p.K, p.N)
-            bytes_per_step += 2 * M * K + 4 * K      # x and gamma once per shared input
-    decode_path = all(mmf.workspace_bytes(M, p.K, p.N) == 0 for p in wl.projections)
+                    calls.append((lib.mmf_bitlinear_fwd_glu,
+                                  (y[jg].data_ptr(), y[ju].data_ptr(), g.data_ptr(), wl.eps,
+                                   self.packed[l, j].data_ptr(), self.scales[l, j].data_ptr(), Mc, p.K, p.N,
+                                   y[j].data_ptr(), self.ws.data_ptr(), self.ws.numel(), self.flags)))
+                    if count:
+                        self.launches_per_step += 1 if mmf.workspace_bytes(Mc, p.K, p.N) == 0 else 2
+                        self.bytes_per_step += p.N * p.K // 4 + 2 * Mc * p.N + 4 + 2 * (2 * Mc * K) + 4 * K
+                        self.ops_per_step += proj_ops(Mc, p.K, p.N)
+                    continue
+                if self.api == "group":
+                    arr = mmf.projection_array([(self.packed[l, j], self.scales[l, j], y[j], wl.projections[j].N)
+                                                for j in js])
+                    self.keep.append(arr)
+                    calls.append((lib.mmf_bitlinear_fwd_group,
+                                  (x.data_ptr(), g.data_ptr(), wl.eps, Mc, K, arr, len(js), self.ws.data_ptr(),
+                                   self.ws.numel(), self.flags)))
+                    if count:
+                        tc = mmf.workspace_bytes(Mc, K, 1) > 0
+                        self.launches_per_step += (1 + len(js)) if tc else 1
+                else:
+                    for j in js:
+                        p = wl.projections[j]
+                        calls.append((lib.mmf_bitlinear_fwd,
+                                      (x.data_ptr(), g.data_ptr(), wl.eps, self.packed[l, j].data_ptr(),
+                                       self.scales[l, j].data_ptr(), Mc, p.K, p.N, y[j].data_ptr(),
+                                       self.ws.data_ptr(), self.ws.numel())))
+                        if count:
+                            self.launches_per_step += 1 if mmf.workspace_bytes(Mc, p.K, p.N) == 0 else 2
+                if count:
+                    for j in js:
+                        p = wl.projections[j]
+                        self.bytes_per_step += p.N * p.K // 4 + 2 * Mc * p.N + 4
+                        self.ops_per_step += proj_ops(Mc, p.K, p.N)
+                    self.bytes_per_step += 2 * Mc * K + 4 * K      # x and gamma once per shared input
+        return calls
 
-    def step(stream_ptr):
+    @staticmethod
+    def run(calls, stream_ptr):
         for f, a in calls:
             rc = f(*a, stream_ptr)
             if rc != 0:
+                from bitlinear_rmsnorm_quant_b200 import mmf
                 raise mmf.MMFError(f.__name__, rc)
 
-    # first calls outside capture (one-time per-device set-up), then capture
-    step(torch.cuda.current_stream().cuda_stream)
-    torch.cuda.synchronize()
-    mmf.check_async()
-    graph = torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream()
-    with torch.cuda.stream(cap):
-        graph.capture_begin()
-        step(cap.cuda_stream)
-        graph.capture_end()
-    torch.cuda.synchronize()
+    def capture(self):
+        # first calls outside capture (one-time per-device set-up), then capture
+        self.run(self.calls, torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        self.mmf.check_async()
+        self.graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        with torch.cuda.stream(cap):
+            self.graph.capture_begin()
+            self.run(self.calls, cap.cuda_stream)
+            self.graph.capture_end()
+        torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
-        graph.replay()
-    torch.cuda.synchronize()
-    mmf.check_async()
+    def time_graph(self, steps, warmup, dist):
+        for _ in range(warmup):
+            self.graph.replay()
+        torch.cuda.synchronize()
+        self.mmf.check_async()
+        clocks = ClockSampler(dist.local_rank)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        torch.cuda.synchronize()
+        clocks.start()
+        e0.record()
+        for _ in range(steps):
+            self.graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        clocks.stop()
+        dist.barrier()
+        self.mmf.check_async()
+        return dist.max(e0.elapsed_time(e1) / steps), clocks.summary()
 
-    # -- timed region: K graph replays, CUDA events on the replay stream
-    clocks = ClockSampler(dist.local_rank)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dist.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    e0.record()
-    for _ in range(args.steps):
-        graph.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    clocks.stop()
-    dist.barrier()
-    ms_local = e0.elapsed_time(e1) / args.steps
-    mmf.check_async()
-    ms = dist.max(ms_local)
+    def time_e2e(self, steps, dist):
+        """End to end through the C ABI with host buffers: every step copies all
+        inputs from pinned host memory to the device and all outputs back.
+        Small steps: one copy in, the graph, one copy out.  Large steps (x + y
+        above E2E_SINGLE_SHOT_BYTES): the tokens stream in E2E_CHUNKS chunks on
+        three streams (copy in, compute, copy out) so the two copy directions
+        and the kernels overlap; host staging is two pinned slots per direction
+        (a chunk's host bytes are its inputs)."""
+        xb, yb = self.x_flat.numel() * 2, self.y_flat.numel() * 2
+        if xb + yb <= E2E_SINGLE_SHOT_BYTES or self.L != 1:
+            h_x = self.x_flat.cpu().pin_memory()
+            h_y = torch.empty(self.y_flat.shape, dtype=torch.bfloat16).pin_memory()
 
-    # -- end to end: pinned host x -> device, the graph (the ABI calls), y -> pinned host
-    h_x = x_flat.cpu().pin_memory()
-    h_y = torch.empty(y_flat.shape, dtype=torch.bfloat16).pin_memory()
+            def e2e_step():
+                self.x_flat.copy_(h_x, non_blocking=True)
+                self.graph.replay()
+                h_y.copy_(self.y_flat, non_blocking=True)
 
-    def e2e_step():
-        x_flat.copy_(h_x, non_blocking=True)
-        graph.replay()
-        h_y.copy_(y_flat, non_blocking=True)
+            n = max(1, min(steps, 200))
+            for _ in range(3):
+                e2e_step()
+            torch.cuda.synchronize()
+            dist.barrier()
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record()
+            for _ in range(n):
+                e2e_step()
+            f1.record()
+            torch.cuda.synchronize()
+            dist.barrier()
+            ms = dist.max(f0.elapsed_time(f1) / n)
+            del h_x, h_y
+            return ms, n, {"mode": "one copy in, the step's graph, one copy out"}
+        wl, M = self.wl, self.wl.M
+        C = E2E_CHUNKS
+        bounds = [(M * i // C, M * (i + 1) // C) for i in range(C)]
+        xin = [(idx, self.xs[0, idx]) for idx, _ in wl.inputs()]
+        outs = [(j, self.ys[0, j]) for j in range(len(wl.projections))]
+        rows = bounds[0][1] - bounds[0][0]
+        h_x = [{idx: t[:rows].cpu().pin_memory() for idx, t in xin} for _ in range(2)]
+        h_y = [{j: torch.empty((rows, t.shape[1]), dtype=torch.bfloat16).pin_memory() for j, t in outs}
+               for _ in range(2)]
+        chunk_calls = [self.make_calls(t0, t1) for t0, t1 in bounds]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        s_cmp = torch.cuda.current_stream()
 
-    e2e_steps = max(1, min(args.steps, 200))
-    for _ in range(3):
+        def e2e_step():
+            # a step's copies in start once the previous step's kernels are done with x
+            s_in.wait_stream(s_cmp)
+            for c, (t0, t1) in enumerate(bounds):
+                n_r = t1 - t0
+                with torch.cuda.stream(s_in):
+                    for idx, t in xin:
+                        t[t0:t1].copy_(h_x[c % 2][idx][:n_r], non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(s_in)
+                s_cmp.wait_event(ev)
+                self.run(chunk_calls[c], s_cmp.cuda_stream)
+                ev2 = torch.cuda.Event()
+                ev2.record(s_cmp)
+                s_out.wait_event(ev2)
+                with torch.cuda.stream(s_out):
+                    for j, t in outs:
+                        h_y[c % 2][j][:n_r].copy_(t[t0:t1], non_blocking=True)
+            ev3 = torch.cuda.Event()
+            ev3.record(s_out)
+            s_cmp.wait_event(ev3)
+
+        n = max(1, min(steps, 5))
         e2e_step()
-    torch.cuda.synchronize()
-    dist.barrier()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record()
-    for _ in range(e2e_steps):
-        e2e_step()
-    f1.record()
-    torch.cuda.synchronize()
-    dist.barrier()
-    e2e_ms = dist.max(f0.elapsed_time(f1) / e2e_steps)
+        torch.cuda.synchronize()
+        dist.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(s_cmp)
+        for _ in range(n):
+            e2e_step()
+        f1.record(s_cmp)
+        torch.cuda.synchronize()
+        dist.barrier()
+        self.mmf.check_async()
+        ms = dist.max(f0.elapsed_time(f1) / n)
+        del h_x, h_y
+        return ms, n, {"mode": f"{C} token chunks streamed on three streams (copy in / kernels / copy out), "
+                               "two pinned host slots per direction"}
 
-    # what every step streams: all layer sets' packed weights, every x, every y
-    streamed = sum(p.N * p.K // 4 for p in wl.projections) * L + 2 * x_flat.numel() + 2 * y_flat.numel()
+
+def run_workload(name, args, dist, steps, warmup, peaks, peak_src, copy_gbs=None, layers=0):
+    """Times one workload's step; returns its JSON object (without cpu_baseline)."""
+    make, default_layers = WORKLOADS[name]
+    wl = make()
+    L = layers or default_layers
+    st = Step(wl, L, dist, args)
+    st.capture()
+    ms, clocks = st.time_graph(steps, warmup, dist)
+    e2e_ms, e2e_steps, e2e_mode = st.time_e2e(steps, dist)
+    M = wl.M
+    streamed = sum(p.N * p.K // 4 for p in wl.projections) * L + 2 * st.x_flat.numel() + 2 * st.y_flat.numel()
     l2_note = (f"inputs larger than L2: {streamed / 1e6:.0f} MB of packed weights, x and y per step > 126 MB"
                if streamed > L2_BYTES else
                f"working set below L2 ({streamed / 1e6:.1f} MB per step, not flushed): a parity-size run, "
@@ -555,72 +683,75 @@ def run_ours(args, dist: Dist):
     tokens_per_step = M * L * dist.world
     value = tokens_per_step / (ms / 1e3)
     e2e_value = tokens_per_step / (e2e_ms / 1e3)
-
-    peaks, peak_src = load_peaks()
-    # the captures are of the default launch configuration (grouped calls, no GLU)
-    traffic = NCU_TRAFFIC.get(wl.name) if args.layers == 0 and args.api == "group" and not args.glu else None
-    if decode_path:
-        achieved = bytes_per_step / (ms / 1e3) / 1e9
+    tc_path = any(st.mmf.workspace_bytes(M, p.K, p.N) > 0 for p in wl.projections)
+    kernel = "gemm_tc_kernel" if tc_path else "gemv_kernel"
+    if hbm_bound(wl):
+        achieved = st.bytes_per_step / (ms / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "kernel": "gemv_kernel",
-                "traffic": traffic["bytes_per_launch"] if traffic else None,
-                "traffic_source": traffic["source"] if traffic else None,
-                "algorithmic_bytes_per_launch": round(bytes_per_step / launches_per_step),
+                "frac": round(achieved / peak, 4), "kernel": kernel, "traffic": None,
+                "algorithmic_bytes_per_launch": round(st.bytes_per_step / st.launches_per_step),
+                "algorithmic_bytes_per_step": st.bytes_per_step,
                 "peak_source": f"{peak_src} hbm_gbs (copy of 1 Gi bf16, read+write bytes)",
-                "algorithmic_bytes_per_step": bytes_per_step,
-                "note": "every launch of the step is this kernel: achieved = bytes per launch / "
-                        "(step time / launches), inter-kernel gaps included"}
+                "note": "achieved = algorithmic bytes per step (packed weights, x and gamma once per shared "
+                        "input, y) / step time: inter-kernel gaps included; traffic: the ncu DRAM counters "
+                        "of this kernel are in the profiles, not measured in this run"}
+        if copy_gbs:
+            roof["copy_kernel_gbs"] = copy_gbs
+            roof["frac_of_copy_kernel"] = round(achieved / copy_gbs, 4)
     else:
-        achieved = ops_per_step / (ms / 1e3) / 1e12
-        # burst peak for a short timed region, sustained (power-capped) for one of seconds
-        long_region = ms * args.steps > 1000.0 and "bf16_tflops_sustained" in peaks
-        peak_key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+        achieved = st.ops_per_step / (ms / 1e3) / 1e12
+        # burst peak for a short step, sustained (power-capped) for a step of many ms
+        long_step = (ms > 10.0 or ms * steps > 1000.0) and "bf16_tflops_sustained" in peaks
+        peak_key = "bf16_tflops_sustained" if long_step else "bf16_tflops"
         peak = float(peaks[peak_key]) * INT8_PER_BF16
+        burst = float(peaks["bf16_tflops"]) * INT8_PER_BF16
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "kernel": "gemm_tc_kernel",
-                "traffic": traffic["bytes_per_launch"] if traffic else None,
-                "traffic_source": traffic["source"] if traffic else None,
+                "frac": round(achieved / peak, 4), "frac_of_burst": round(achieved / burst, 4),
+                "frac_of_datasheet_4500": round(achieved / 4500.0, 4),
+                "kernel": kernel, "traffic": None,
                 "peak_source": f"{peak_src} {peak_key} x {INT8_PER_BF16} (nominal int8:bf16 dense ratio)",
-                "library_int8_tops": library_int8_tops(),
-                "algorithmic_ops_per_step": ops_per_step,
-                "note": "int8 TOPS over the whole step (quantiser kernel included)"}
-
-    result = {
-        "metric": METRIC,
-        "value": round(value, 2),
+                "algorithmic_ops_per_step": st.ops_per_step,
+                "note": "int8 TOPS over the whole step (quantiser kernels included); traffic: the ncu DRAM "
+                        "counters of this kernel are in the profiles, not measured in this run"}
+    res = {
+        "metric": METRIC, "value": round(value, 2),
         "unit": "tokens/s (one token through one BitLinear layer set)",
-        "n_gpus": dist.world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": round(ms, 6),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "int8",
+        "n_gpus": dist.world, "steps": steps, "warmup": warmup, "ms_per_step": round(ms, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic (seeded SplitMix64/Box-Muller; random-init latent weights)",
         "config": {
             "workload": wl.name, "description": wl.description, "M": M, "layer_sets": L,
             "projections": [f"{p.K}->{p.N}" for p in wl.projections],
             "packed_weight_bytes": sum(p.N * p.K // 4 for p in wl.projections) * L,
-            "l2": l2_note,
-            "graph": "one CUDA graph per step", "parallelism": f"dp{dist.world} (token-parallel replicas)",
+            "l2": l2_note, "graph": "one CUDA graph per step",
+            "parallelism": f"dp{dist.world} (token-parallel replicas)",
             "api": "mmf_bitlinear_fwd_group" if args.api == "group" else "mmf_bitlinear_fwd",
-            "pdl": not args.no_pdl and args.api == "group", "launches_per_step": launches_per_step,
+            "pdl": not args.no_pdl and args.api == "group", "launches_per_step": st.launches_per_step,
             "glu_down": bool(args.glu),
         },
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s (one token through one BitLinear layer set)",
-                "h2d_bytes_per_step": int(h_x.numel() * 2), "d2h_bytes_per_step": int(h_y.numel() * 2),
-                "steps": e2e_steps},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks.summary(),
+                "h2d_bytes_per_step": int(st.x_flat.numel() * 2), "d2h_bytes_per_step": int(st.y_flat.numel() * 2),
+                "steps": e2e_steps, **e2e_mode},
+        "gpu_launches": st.launches_per_step * steps,
+        "clocks": clocks,
     }
-    del graph
-    return result, wl, L
+    st.graph = None
+    del st
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res, wl
 
 
 # ----------------------------------------------------------------------------- oracle timing
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
 
 def time_oracle(wl, sample_tokens: int | None, budget_s: float, max_reps: int | None = None,
                 one_projection_per_rep: bool = False):
@@ -657,8 +788,7 @@ def time_oracle(wl, sample_tokens: int | None, budget_s: float, max_reps: int | 
         if time.perf_counter() - t_start > budget_s and all(per_proj):
             break
     t_set = sum(statistics.median(v) for v in per_proj)
-    threads = min(orc.num_threads(), M)
-    return M / t_set, M, threads, reps
+    return M / t_set, M, orc.num_threads(), reps
 
 
 def oracle_sample_tokens(wl, cap):
@@ -669,9 +799,10 @@ def cpu_baseline_obj(wl, budget_s=12.0):
     sample = oracle_sample_tokens(wl, 512)
     tps, M, threads, reps = time_oracle(wl, sample, budget_s)
     return {"value": round(tps, 3), "unit": "tokens/s (one token through one BitLinear layer set)",
-            "cores": threads, "kind": "oracle",
-            "sample": f"{M} tokens x all {len(wl.projections)} projections, median of {reps} rep(s), "
-                      f"OpenMP over tokens; weights ternarised untimed"
+            "cores": threads, "threads": threads, "host_cores": host_cores(), "kind": "oracle",
+            "sample": f"{M} tokens x all {len(wl.projections)} projections, median of {reps} rep(s); the "
+                      f"contraction on OpenMP threads over (token, output row) pairs, normalisation and "
+                      f"rescale on one thread; weights ternarised untimed"
                       + (f"; extrapolated linearly from {M} of {wl.M} tokens" if M < wl.M else "")}
 
 
@@ -697,8 +828,9 @@ def run_reference(args, dist: Dist):
         "config": {"workload": wl.name, "description": wl.description, "M": wl.M,
                    "projections": [f"{p.K}->{p.N}" for p in wl.projections]},
         "cpu_baseline": {"value": round(tps, 3), "unit": "tokens/s (one token through one BitLinear layer set)",
-                         "cores": threads, "kind": "oracle",
-                         "sample": f"{M} tokens; each step one projection (round robin); wall {wall:.1f} s"},
+                         "cores": threads, "threads": threads, "host_cores": host_cores(), "kind": "oracle",
+                         "sample": f"{M} tokens; each step one projection (round robin); wall {wall:.1f} s"
+                                   + (f"; extrapolated linearly from {M} of {wl.M} tokens" if M < wl.M else "")},
         "e2e": {"value": round(tps, 3), "unit": "tokens/s (one token through one BitLinear layer set)",
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -709,12 +841,18 @@ def run_reference(args, dist: Dist):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--layers", type=int, default=0, help="layer sets per step (default per workload)")
+    ap.add_argument("--secondary", default=None,
+                    help="comma-separated workloads timed after the main one in the same run, or 'none' "
+                         f"(default with the default workload: {DEFAULT_SECONDARY}; otherwise none)")
+    ap.add_argument("--secondary-min-steps", type=int, default=200,
+                    help="timed steps of each secondary workload: max(--steps, this)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-copy-kernel", action="store_true", help="skip timing mmf_hbm_copy")
     ap.add_argument("--api", choices=("group", "single"), default="group",
                     help="group: one call per set of projections sharing x; single: one call per projection")
     ap.add_argument("--glu", action="store_true",
@@ -723,6 +861,12 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.secondary is None:
+        args.secondary = DEFAULT_SECONDARY if args.workload == DEFAULT_WORKLOAD else "none"
+    secondary = [] if args.secondary in ("", "none") else args.secondary.split(",")
+    for w in secondary:
+        if w not in WORKLOADS or WORKLOADS[w][0] is None:
+            raise SystemExit(f"--secondary: unknown forward workload {w}")
     dist = Dist(args.gpus)
     try:
         if args.impl == "reference" and args.workload == "mlgru-scan-1.3b":
@@ -750,12 +894,27 @@ def main(argv=None):
             return 0
         if not torch.cuda.is_available():
             raise SystemExit("bench.py --impl ours needs a CUDA device")
+        torch.cuda.set_device(dist.local_rank)
         if args.workload in ("mlgru-scan-1.3b", "bwd-prefill-1.3b"):
             res = run_scan(args, dist) if args.workload == "mlgru-scan-1.3b" else run_bwd(args, dist)
             if dist.rank == 0:
                 print(json.dumps(res), flush=True)
             return 0
-        res, wl, L = run_ours(args, dist)
+        peaks, peak_src = load_peaks()
+        copy = None if args.no_copy_kernel else time_hbm_copy(torch.device("cuda", dist.local_rank))
+        copy_gbs = copy["gbs"] if copy else None
+        res, wl = run_workload(args.workload, args, dist, args.steps, args.warmup, peaks, peak_src, copy_gbs,
+                               layers=args.layers)
+        if copy:
+            res["hbm_copy"] = copy
+        sec = []
+        for w in secondary:
+            r, _ = run_workload(w, args, dist, max(args.steps, args.secondary_min_steps), args.warmup, peaks,
+                                peak_src, copy_gbs)
+            sec.append({k: r[k] for k in ("value", "unit", "ms_per_step", "steps", "warmup", "roofline", "e2e",
+                                          "gpu_launches", "clocks", "config")})
+        if sec:
+            res["secondary"] = sec
         if dist.rank == 0:
             if dist.world == 1 and not args.no_cpu_baseline:
                 res["cpu_baseline"] = cpu_baseline_obj(wl)

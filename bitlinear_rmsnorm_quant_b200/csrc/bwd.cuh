@@ -1,67 +1,19 @@
-// bwd.cuh -- backward of the fused BitLinear layer with the straight-through
-// estimator (ld246.com, section "训练与优化：新的策略": the non-differentiable
-// ternary weights and quantisation are back-propagated with a surrogate
-// gradient, read as passing gradients through the quantisers unchanged).
-// With x_q = q * (absmax / 127) and W_q = w~ * beta the forward is
-// y = x_q . W_q^T, so
+// bwd.cuh -- the parts of the straight-through backward of the fused
+// BitLinear layer around its two products (ld246.com, section "训练与优化：新的
+// 策略": the non-differentiable ternary weights and quantisation are
+// back-propagated with a surrogate gradient, read as passing gradients through
+// the quantisers unchanged).  With x_q = q * (absmax / 127) and
+// W_q = w~ * beta the forward is y = x_q . W_q^T, so
 //   dr = dy . W_q            (the gradient at the normalised activations)
 //   dW = dy^T . x_q          (the gradient at the latent weights)
-// and RMSNorm's backward gives dx and dgamma from dr.  The two products are
-// plain bf16 GEMMs (cuBLAS, fp32 accumulation) over operands these kernels
-// prepare: w~ as bf16 {-1, 0, +1} (beta is applied to dr afterwards, exactly),
-// q as bf16 (exact) and dy * absmax / 127 rounded to bf16.
+// (both on the tensor cores, bwd_tc.cuh), and RMSNorm's backward gives dx and
+// dgamma from dr (here).
 #pragma once
 #include "common.cuh"
 
 namespace mmf {
 
 constexpr int kBwdThreads = 256;
-
-// w~ as bf16 from the packed codes: one thread per 32-bit word (16 weights)
-__global__ void __launch_bounds__(kBwdThreads) unpack_ternary_bf16_kernel(const uint32_t* __restrict__ packed,
-                                                                          int64_t nwords,
-                                                                          uint16_t* __restrict__ wb) {
-    const int64_t i = static_cast<int64_t>(blockIdx.x) * kBwdThreads + threadIdx.x;
-    if (i >= nwords) return;
-    const uint32_t w = __ldg(packed + i);
-    // weight j of the group: code at bits 8 (j % 4) + 2 (j / 4); bf16 of c - 1
-    uint32_t out[8];
-#pragma unroll
-    for (int j2 = 0; j2 < 8; ++j2) {
-        uint32_t pair = 0;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int j = 2 * j2 + h;
-            const uint32_t c = (w >> (8 * (j & 3) + 2 * (j >> 2))) & 3u;
-            const uint32_t bits = c == 0 ? 0xBF80u : (c == 2 ? 0x3F80u : 0u);  // -1, +1, 0
-            pair |= bits << (16 * h);
-        }
-        out[j2] = pair;
-    }
-    uint4* dst = reinterpret_cast<uint4*>(wb + 16 * i);
-    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-}
-
-// dy * (absmax / 127) as bf16 (the left operand of dW), one thread per element
-__global__ void __launch_bounds__(kBwdThreads) scale_dy_kernel(const uint16_t* __restrict__ dy,
-                                                               const float* __restrict__ absmax, int64_t M, int64_t N,
-                                                               uint16_t* __restrict__ dys) {
-    const int64_t i = static_cast<int64_t>(blockIdx.x) * kBwdThreads + threadIdx.x;
-    if (i >= M * N) return;
-    const int64_t m = i / N;
-    const float s = __fdiv_rn(__ldg(absmax + m), 127.0f);
-    const float v = __fmul_rn(__uint_as_float(static_cast<uint32_t>(__ldg(dy + i)) << 16), s);
-    dys[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-}
-
-// q as bf16 (exact for |q| <= 127), one thread per element
-__global__ void __launch_bounds__(kBwdThreads) codes_bf16_kernel(const int8_t* __restrict__ q, int64_t n,
-                                                                 uint16_t* __restrict__ qb) {
-    const int64_t i = static_cast<int64_t>(blockIdx.x) * kBwdThreads + threadIdx.x;
-    if (i >= n) return;
-    qb[i] = __bfloat16_as_ushort(__float2bfloat16_rn(static_cast<float>(__ldg(q + i))));
-}
 
 // RMSNorm backward for one token row per CTA: with g_k = beta * dr_k,
 //   dx_k = inv gamma_k g_k - x_k inv^3 (sum_j gamma_j g_j x_j) / K

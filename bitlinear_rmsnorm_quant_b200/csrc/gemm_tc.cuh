@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 qsum_s[i] = qs;
                 cm_s[i] = cm;
             }
-            // the four warps leave together or not at all (they share named barriers)
+            // the epilogue warps leave together or not at all (they share a named barrier)
             const bool got = mbar_wait(&tfull_bar[buf], (li >> 1) & 1, &abort_flag);
             if (!named_barrier_and<kTcEpiBarrier, kTcEpiWarps * 32>(got)) break;
             tc_fence_after();

@@ -3,9 +3,7 @@
 // the headers included below; this is the only translation unit.
 #include "mmf.h"
 
-#include <cublas_v2.h>
 #include <cudaTypedefs.h>
-#include <dlfcn.h>
 
 #include <mutex>
 #include <utility>
@@ -14,10 +12,12 @@
 #include "copy.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_tc.cuh"
 #include "pack.cuh"
 #include "quant.cuh"
 #include "scan.cuh"
 #include "bwd.cuh"
+#include "bwd_tc.cuh"
 
 namespace {
 
@@ -30,21 +30,7 @@ constexpr int64_t kMaxK = 65536;  // the quantiser stages one bf16 row (2K bytes
 struct DeviceState {
     bool ready = false;
     int num_sms = 0;
-    cublasHandle_t cublas = nullptr;  // backward only, created on first use
 };
-
-// cuBLAS serves the backward's two plain bf16 GEMMs only; it is opened on the
-// first backward call, so the forward path never depends on it.
-using CublasGemmExFn = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int,
-                                          const void*, const void*, cudaDataType, int, const void*, cudaDataType, int,
-                                          const void*, void*, cudaDataType, int, cublasComputeType_t, cublasGemmAlgo_t);
-struct CublasApi {
-    decltype(&cublasCreate_v2) create = nullptr;
-    decltype(&cublasSetStream_v2) set_stream = nullptr;
-    CublasGemmExFn gemm = nullptr;
-    bool tried = false;
-};
-CublasApi g_cublas;
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -110,6 +96,10 @@ mmf_status device_state(DeviceState** out) {
         if (e == cudaSuccess) e = set_tc_attrs<64>();
         if (e == cudaSuccess) e = set_tc_attrs<128>();
         if (e == cudaSuccess) e = set_tc_attrs<256>();
+        if (e == cudaSuccess) e = set_smem(gemv_tc_kernel<16, true>, kGtSmemBudget);
+        if (e == cudaSuccess) e = set_smem(gemv_tc_kernel<16, false>, kGtSmemBudget);
+        if (e == cudaSuccess) e = set_smem(gemv_tc_kernel<32, true>, kGtSmemBudget);
+        if (e == cudaSuccess) e = set_smem(gemv_tc_kernel<32, false>, kGtSmemBudget);
         if (e == cudaSuccess) e = set_gemv_attrs<1>();
         if (e == cudaSuccess) e = set_gemv_attrs<2>();
         if (e == cudaSuccess) e = set_gemv_attrs<3>();
@@ -118,11 +108,10 @@ mmf_status device_state(DeviceState** out) {
         if (e == cudaSuccess) e = set_gemv_attrs<6>();
         if (e == cudaSuccess) e = set_gemv_attrs<7>();
         if (e == cudaSuccess) e = set_gemv_attrs<8>();
-        // both buffer counts may be asked about up to the streaming kernel's limit
-        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_stream_kernel<1>, quant_stream_smem(kMaxQuantStreamK, 1));
-        if (e == cudaSuccess) e = set_smem(rmsnorm_quant_stream_kernel<2>, quant_stream_smem(kMaxQuantStreamK, 1));
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8>, 2 * kMaxK);  // one row of the largest K
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8, true>, 2 * kMaxK);
+        if (e == cudaSuccess) e = set_smem(gemm_bwd_kernel<0>, BwLayout<0>::smem_bytes);
+        if (e == cudaSuccess) e = set_smem(gemm_bwd_kernel<1>, BwLayout<1>::smem_bytes);
         if (e != cudaSuccess) return MMF_ERR_CUDA;
         if (!g_encode_tiled) {
             void* fn = nullptr;
@@ -149,9 +138,24 @@ mmf_status check_shape(int64_t M, int64_t K, int64_t N) {
     return MMF_OK;
 }
 
+// Small M: up to kDecodeTcMinM - 1 tokens the CUDA-core decode kernel (its
+// add/sub cost grows with M); from there to kDecodeTcMaxM the decode
+// tensor-core kernel after a quantiser launch; beyond, the large-M path.
+constexpr int64_t kDecodeTcMinM = 2;
+constexpr int64_t kDecodeTcMaxM = 32;
+
 bool takes_gemv(int64_t M, int64_t K) {
+    if (M >= kDecodeTcMinM) return false;
     GemvPlan plan;
     return gemv_plan(static_cast<int>(M), static_cast<int>(K), 1, 148, &plan);
+}
+
+int decode_tc_nt(int64_t M) { return M <= 16 ? 16 : 32; }
+
+bool takes_decode_tc(int64_t M, int64_t K) {
+    if (M < kDecodeTcMinM || M > kDecodeTcMaxM) return false;
+    GemvTcPlan plan;
+    return gemv_tc_plan(decode_tc_nt(M), static_cast<int>(K), 1, 148, &plan);
 }
 
 // Launches a kernel, as a programmatic dependent of the previous kernel on the
@@ -194,6 +198,21 @@ size_t workspace_size_tc(int64_t M, int64_t K) {
     return align256(static_cast<size_t>(M) * K) + 2 * align256(4 * static_cast<size_t>(M));
 }
 
+// decode tensor-core path: the codes in the B layout of NT rows, absmax, qsum
+size_t workspace_size_dtc(int64_t M, int64_t K) {
+    return align256(static_cast<size_t>(decode_tc_nt(M)) * K) + 2 * align256(4 * static_cast<size_t>(M));
+}
+
+Workspace carve_dtc(void* ws, int64_t M, int64_t K) {
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    const size_t cb = align256(static_cast<size_t>(decode_tc_nt(M)) * K);
+    Workspace w;
+    w.q = reinterpret_cast<int8_t*>(b);
+    w.absmax = reinterpret_cast<float*>(b + cb);
+    w.qsum = reinterpret_cast<int*>(b + cb + align256(4 * static_cast<size_t>(M)));
+    return w;
+}
+
 Workspace carve(void* ws, int64_t M, int64_t K) {
     uint8_t* b = static_cast<uint8_t*>(ws);
     Workspace w;
@@ -224,6 +243,20 @@ mmf_status make_maps(const int8_t* q, const uint32_t* packed, int64_t M, int64_t
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MMF_ERR_CUDA;
     }
+    return MMF_OK;
+}
+
+// A 2D tensor map over a row-major [rows][cols] array of `esize`-byte elements
+// with row pitch `pitch` bytes (a multiple of 16), box {box_cols, box_rows}.
+mmf_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t cols, int64_t rows,
+                     int64_t pitch, int box_cols, int box_rows, CUtensorMapSwizzle swz) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pitch)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t es[2] = {1, 1};
+    if (g_encode_tiled(map, dtype, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MMF_ERR_CUDA;
     return MMF_OK;
 }
 
@@ -271,34 +304,43 @@ mmf_status launch_gemv(const GemvParams& p, const GemvPlan& plan, cudaStream_t s
     }
 }
 
+// bl_nt > 0: codes in the decode tensor-core kernel's B layout of bl_nt rows
+template <bool FUSED>
+mmf_status launch_gemv_tc(int NT, const GemvTcParams& p, const GemvTcPlan& plan, cudaStream_t s) {
+    // a programmatic dependent of the quantiser launched just before it: only
+    // the packed weights and scales (parameters) are read before the wait
+    const dim3 grid(static_cast<unsigned>(plan.grid));
+    if (NT == 16) return launch(gemv_tc_kernel<16, FUSED>, grid, dim3(kGtThreads), plan.smem_bytes, s, true, p);
+    return launch(gemv_tc_kernel<32, FUSED>, grid, dim3(kGtThreads), plan.smem_bytes, s, true, p);
+}
+
 mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K, int8_t* q,
                         float* absmax, int* qsum, cudaStream_t s, bool pdl, int num_sms,
-                        const uint16_t* u = nullptr) {
+                        const uint16_t* u = nullptr, int bl_nt = 0) {
+    const dim3 rows_grid(static_cast<unsigned>(bl_nt > 0 ? bl_nt : M));
     if (u)  // GLU: one CTA of 8 warps per row, forming SiLU(g) * u on the way
-        return launch(rmsnorm_quant_kernel<8, true>, dim3(static_cast<unsigned>(M)), dim3(256),
-                      static_cast<size_t>(K) * 2, s, pdl, x, gamma, eps, static_cast<int>(K), M, q, absmax, qsum, u);
-    if (M < kQuantWarpRowMinM || K > kMaxQuantStreamK)  // one CTA of 8 warps per row
-        return launch(rmsnorm_quant_kernel<8>, dim3(static_cast<unsigned>(M)), dim3(256), static_cast<size_t>(K) * 2,
-                      s, pdl, x, gamma, eps, static_cast<int>(K), M, q, absmax, qsum, static_cast<const uint16_t*>(nullptr));
-    // persistent: as many CTAs as fit on the SMs at once, never more than the
-    // rows need; two row buffers per warp unless that leaves one CTA per SM
-    int per_sm[2] = {0, 0};
-    for (int nb = 1; nb <= 2; ++nb) {
-        const size_t smem = quant_stream_smem(static_cast<int>(K), nb);
-        if (smem > quant_stream_smem(kMaxQuantStreamK, 1)) continue;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                &per_sm[nb - 1], nb == 1 ? rmsnorm_quant_stream_kernel<1> : rmsnorm_quant_stream_kernel<2>,
-                kQuantStreamWarps * 32, smem) != cudaSuccess)
-            return MMF_ERR_CUDA;
-    }
-    const int nb = per_sm[1] >= 2 ? 2 : 1;
-    if (per_sm[nb - 1] < 1) return MMF_ERR_CUDA;
-    int64_t grid = static_cast<int64_t>(per_sm[nb - 1]) * num_sms;
-    const int64_t need = (M + kQuantStreamWarps - 1) / kQuantStreamWarps;
+        return launch(rmsnorm_quant_kernel<8, true>, rows_grid, dim3(256), static_cast<size_t>(K) * 2, s, pdl, x,
+                      gamma, eps, static_cast<int>(K), M, q, absmax, qsum, u, bl_nt);
+    if (bl_nt > 0 || M < kQuantWarpRowMinM || K > kMaxQuantRegK)  // one CTA of 8 warps per row
+        return launch(rmsnorm_quant_kernel<8>, rows_grid, dim3(256), static_cast<size_t>(K) * 2, s, pdl, x, gamma, eps,
+                      static_cast<int>(K), M, q, absmax, qsum, static_cast<const uint16_t*>(nullptr), bl_nt);
+    // persistent: rows in registers, WPR warps per row (K <= 2048 WPR), as many
+    // CTAs as fit on the SMs at once, never more than the rows need
+    const int wpr = static_cast<int>((K + 2047) / 2048);
+    void (*kern)(const uint16_t*, const float*, float, int, int64_t, int8_t*, float*, int*) =
+        wpr == 1 ? rmsnorm_quant_reg_kernel<1>
+                 : (wpr == 2 ? rmsnorm_quant_reg_kernel<2>
+                             : (wpr == 3 ? rmsnorm_quant_reg_kernel<3> : rmsnorm_quant_reg_kernel<4>));
+    const int threads = quant_reg_warps(wpr) * 32;
+    const int rpc = quant_reg_warps(wpr) / wpr;
+    const size_t smem = static_cast<size_t>(K) * 4;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess || per_sm < 1)
+        return MMF_ERR_CUDA;
+    int64_t grid = static_cast<int64_t>(per_sm) * num_sms;
+    const int64_t need = (M + rpc - 1) / rpc;
     if (grid > need) grid = need;
-    const size_t smem = quant_stream_smem(static_cast<int>(K), nb);
-    return launch(nb == 1 ? rmsnorm_quant_stream_kernel<1> : rmsnorm_quant_stream_kernel<2>,
-                  dim3(static_cast<unsigned>(grid)), dim3(kQuantStreamWarps * 32), smem, s, pdl, x, gamma, eps,
+    return launch(kern, dim3(static_cast<unsigned>(grid)), dim3(threads), smem, s, pdl, x, gamma, eps,
                   static_cast<int>(K), M, q, absmax, qsum);
 }
 
@@ -336,6 +378,34 @@ mmf_status fwd_impl(const uint16_t* x, const float* gamma, float eps, int64_t M,
         p.stage_bytes = plan.stage_bytes;
         p.stages = plan.stages;
         return u ? launch_gemv<true, true>(p, plan, s, pdl) : launch_gemv<true>(p, plan, s, pdl);
+    }
+    if (takes_decode_tc(M, K)) {
+        const int NT = decode_tc_nt(M);
+        GemvTcPlan tplan;
+        if (!gemv_tc_plan(NT, static_cast<int>(K), R, dev->num_sms, &tplan)) return MMF_ERR_UNSUPPORTED_SHAPE;
+        Workspace w = carve_dtc(workspace, M, K);
+        mmf_status st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s, pdl, dev->num_sms, u, NT);
+        if (st != MMF_OK) return st;
+        GemvTcParams p{};
+        p.codes = w.q;
+        p.absmax = w.absmax;
+        p.qsum = w.qsum;
+        int g = 0;
+        p.row_start[0] = 0;
+        for (int i = 0; i < count; ++i) {
+            if (proj[i].N == 0) continue;
+            p.packed[g] = proj[i].packed;
+            p.scale[g] = proj[i].scale;
+            p.y[g] = proj[i].y;
+            p.row_start[g + 1] = p.row_start[g] + static_cast<int>(proj[i].N);
+            ++g;
+        }
+        p.nproj = g;
+        p.M = static_cast<int>(M);
+        p.K = static_cast<int>(K);
+        p.rows_per_cta = tplan.rows_per_cta;
+        p.b_slots = tplan.b_slots;
+        return launch_gemv_tc<true>(NT, p, tplan, s);
     }
     Workspace w = carve(workspace, M, K);
     mmf_status st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s, pdl, dev->num_sms, u);
@@ -385,6 +455,7 @@ size_t mmf_packed_bytes(int64_t N, int64_t K) {
 size_t mmf_workspace_bytes(int64_t M, int64_t K, int64_t N) {
     if (check_shape(M, K, N) != MMF_OK || M == 0 || N == 0) return 0;
     if (takes_gemv(M, K)) return 0;
+    if (takes_decode_tc(M, K)) return workspace_size_dtc(M, K);
     return workspace_size_tc(M, K);
 }
 
@@ -458,9 +529,31 @@ int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t 
         p.stages = plan.stages;
         return launch_gemv<false>(p, plan, s, false);
     }
+    if (takes_decode_tc(M, K)) {
+        const int NT = decode_tc_nt(M);
+        GemvTcPlan tplan;
+        if (!gemv_tc_plan(NT, static_cast<int>(K), N, dev->num_sms, &tplan)) return MMF_ERR_UNSUPPORTED_SHAPE;
+        Workspace w = carve_dtc(workspace, M, K);
+        st = launch(qsum_kernel, dim3(static_cast<unsigned>(NT)), dim3(kQuantThreads), 0, s, false, q,
+                    static_cast<int>(K), M, w.qsum, w.q, NT);
+        if (st != MMF_OK) return st;
+        GemvTcParams p{};
+        p.codes = w.q;
+        p.qsum = w.qsum;
+        p.packed[0] = packed;
+        p.acc = acc;
+        p.row_start[0] = 0;
+        p.row_start[1] = static_cast<int>(N);
+        p.nproj = 1;
+        p.M = static_cast<int>(M);
+        p.K = static_cast<int>(K);
+        p.rows_per_cta = tplan.rows_per_cta;
+        p.b_slots = tplan.b_slots;
+        return launch_gemv_tc<false>(NT, p, tplan, s);
+    }
     Workspace w = carve(workspace, M, K);
     st = launch(qsum_kernel, dim3(static_cast<unsigned>(M)), dim3(kQuantThreads), 0, s, false, q, static_cast<int>(K),
-                w.qsum);
+                M, w.qsum, static_cast<int8_t*>(nullptr), 0);
     if (st != MMF_OK) return st;
     TcParams p{};
     p.qsum = w.qsum;
@@ -496,10 +589,10 @@ int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps, const ui
 
 size_t mmf_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N) {
     if (check_shape(M, K, N) != MMF_OK) return 0;
-    const size_t m = static_cast<size_t>(M), k = static_cast<size_t>(K), n = static_cast<size_t>(N);
+    const size_t m = static_cast<size_t>(M), k = static_cast<size_t>(K);
     const size_t chunks = (m + kDgammaRows - 1) / kDgammaRows;
-    return align256(m * k) + 3 * align256(4 * m) + align256(2 * n * k) + align256(2 * m * n) + align256(2 * m * k) +
-           align256(4 * m * k) + align256(8 * chunks * k);
+    // q, absmax, qsum, inv, dr (fp32), dgamma partials (fp64)
+    return align256(m * k) + 3 * align256(4 * m) + align256(4 * m * k) + align256(8 * chunks * k);
 }
 
 int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma, float eps, const uint32_t* packed,
@@ -508,11 +601,14 @@ int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma,
     if (!(eps >= 0.0f) || eps > 1e30f) return MMF_ERR_INVALID_ARG;
     mmf_status st = check_shape(M, K, N);
     if (st != MMF_OK) return st;
-    // 32-bit GEMM sizes; the dgamma row chunks on grid.y
-    if (M > 65535L * kDgammaRows || N * M > kMaxDim || M * K > kMaxDim) return MMF_ERR_UNSUPPORTED_SHAPE;
+    // dy rows are read by TMA (row pitch a multiple of 16 bytes); the dgamma row chunks on grid.y
+    if ((N % 8) != 0 || M > 65535L * kDgammaRows) return MMF_ERR_UNSUPPORTED_SHAPE;
     if (M == 0 && N == 0) return MMF_OK;
-    if (!dy || !x || !gamma || !packed || !scale || !dx || !dgamma || !dW || !workspace)
-        return MMF_ERR_INVALID_ARG;
+    // buffers of an empty extent may be NULL
+    if (!gamma || !scale || !dgamma) return MMF_ERR_INVALID_ARG;
+    if (M > 0 && (!x || !dx || !workspace)) return MMF_ERR_INVALID_ARG;
+    if (N > 0 && !dW) return MMF_ERR_INVALID_ARG;
+    if (M > 0 && N > 0 && (!dy || !packed)) return MMF_ERR_INVALID_ARG;
     if (!aligned16(dy) || !aligned16(x) || !aligned16(gamma) || !aligned16(packed) || !aligned16(scale) ||
         !aligned16(dx) || !aligned16(dgamma) || !aligned16(dW) || !aligned16(workspace))
         return MMF_ERR_MISALIGNED;
@@ -520,23 +616,9 @@ int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma,
     DeviceState* dev;
     if ((st = device_state(&dev)) != MMF_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    {
-        std::lock_guard<std::mutex> lock(g_mu);
-        if (!g_cublas.tried) {
-            g_cublas.tried = true;
-            void* h = dlopen("libcublas.so.12", RTLD_NOW | RTLD_LOCAL);
-            if (h) {
-                g_cublas.create = reinterpret_cast<decltype(&cublasCreate_v2)>(dlsym(h, "cublasCreate_v2"));
-                g_cublas.set_stream = reinterpret_cast<decltype(&cublasSetStream_v2)>(dlsym(h, "cublasSetStream_v2"));
-                g_cublas.gemm = reinterpret_cast<CublasGemmExFn>(dlsym(h, "cublasGemmEx"));
-            }
-        }
-        if (!g_cublas.create || !g_cublas.set_stream || !g_cublas.gemm) return MMF_ERR_CUDA;
-        if (!dev->cublas && g_cublas.create(&dev->cublas) != CUBLAS_STATUS_SUCCESS) return MMF_ERR_CUDA;
-    }
-    // workspace: q, absmax, qsum, inv, w~ (bf16), dy * absmax / 127 (bf16), q (bf16), dr (fp32)
+    // workspace: q, absmax, qsum, inv, dr (fp32 [M][K]), dgamma partials
     uint8_t* b = static_cast<uint8_t*>(workspace);
-    const size_t m = static_cast<size_t>(M), k = static_cast<size_t>(K), n = static_cast<size_t>(N);
+    const size_t m = static_cast<size_t>(M), k = static_cast<size_t>(K);
     int8_t* q = reinterpret_cast<int8_t*>(b);
     b += align256(m * k);
     float* absmax = reinterpret_cast<float*>(b);
@@ -545,44 +627,64 @@ int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma,
     b += align256(4 * m);
     float* inv = reinterpret_cast<float*>(b);
     b += align256(4 * m);
-    uint16_t* wb = reinterpret_cast<uint16_t*>(b);
-    b += align256(2 * n * k);
-    uint16_t* dys = reinterpret_cast<uint16_t*>(b);
-    b += align256(2 * m * n);
-    uint16_t* qb = reinterpret_cast<uint16_t*>(b);
-    b += align256(2 * m * k);
     float* dr = reinterpret_cast<float*>(b);
     b += align256(4 * m * k);
     double* part = reinterpret_cast<double*>(b);
     const int chunks = static_cast<int>((M + kDgammaRows - 1) / kDgammaRows);
+    const int row_tiles = static_cast<int>(K / kBwRows);
 
     if (M > 0 && (st = launch_quant(x, gamma, eps, M, K, q, absmax, qsum, s, false, dev->num_sms)) != MMF_OK) return st;
-    const auto blocks = [](int64_t count) { return dim3(static_cast<unsigned>((count + kBwdThreads - 1) / kBwdThreads)); };
-    if (N > 0 && (st = launch(unpack_ternary_bf16_kernel, blocks(N * K / 16), dim3(kBwdThreads), 0, s, false, packed,
-                              N * K / 16, wb)) != MMF_OK)
-        return st;
-    if (M > 0 && N > 0 &&
-        (st = launch(scale_dy_kernel, blocks(M * N), dim3(kBwdThreads), 0, s, false, dy, absmax, M, N, dys)) != MMF_OK)
-        return st;
-    if (M > 0 && (st = launch(codes_bf16_kernel, blocks(M * K), dim3(kBwdThreads), 0, s, false, q, M * K, qb)) != MMF_OK)
-        return st;
-    if (g_cublas.set_stream(dev->cublas, s) != CUBLAS_STATUS_SUCCESS) return MMF_ERR_CUDA;
-    const float one = 1.0f, zero = 0.0f;
-    // dr[M][K] = dy[M][N] . w~[N][K]   (column-major: dr^T = w~^T dy^T)
-    if (M > 0 && g_cublas.gemm(dev->cublas, CUBLAS_OP_N, CUBLAS_OP_N, static_cast<int>(K), static_cast<int>(M),
-                               static_cast<int>(N), &one, wb, CUDA_R_16BF, static_cast<int>(K), dy, CUDA_R_16BF,
-                               static_cast<int>(N), &zero, dr, CUDA_R_32F, static_cast<int>(K), CUBLAS_COMPUTE_32F,
-                               CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-        return MMF_ERR_CUDA;
-    // dW[N][K] = dys^T[N][M] . q[M][K]   (column-major: dW^T = q^T dys)
-    if (N > 0 && g_cublas.gemm(dev->cublas, CUBLAS_OP_N, CUBLAS_OP_T, static_cast<int>(K), static_cast<int>(N),
-                               static_cast<int>(M), &one, qb, CUDA_R_16BF, static_cast<int>(K), dys, CUDA_R_16BF,
-                               static_cast<int>(N), &zero, dW, CUDA_R_32F, static_cast<int>(K), CUBLAS_COMPUTE_32F,
-                               CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-        return MMF_ERR_CUDA;
+    // dr[M][K] = dy . w~ (an empty contraction when N == 0 gives zeros)
+    if (M > 0 && N == 0) {
+        if (cudaMemsetAsync(dr, 0, 4 * m * k, s) != cudaSuccess) return MMF_ERR_CUDA;
+    } else if (M > 0) {
+        CUtensorMap mb, mr;
+        if ((st = encode_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy, N, M, 2 * N, kBwKs, kBwCols,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) != MMF_OK)
+            return st;
+        if ((st = encode_2d(&mr, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, K / 4, N, K / 4, kBwRows / 4, kBwKs,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)) != MMF_OK)
+            return st;
+        BwParams bp{};
+        bp.out = dr;
+        bp.K = static_cast<int>(K);
+        bp.cols = static_cast<int>(M);
+        bp.contr = static_cast<int>(N);
+        bp.row_tiles = row_tiles;
+        bp.num_tiles = row_tiles * static_cast<int>((M + kBwCols - 1) / kBwCols);
+        const dim3 grid(static_cast<unsigned>(bp.num_tiles < dev->num_sms ? bp.num_tiles : dev->num_sms));
+        if ((st = launch(gemm_bwd_kernel<0>, grid, dim3(kBwThreads), BwLayout<0>::smem_bytes, s, false, mb, mr, bp)) !=
+            MMF_OK)
+            return st;
+    }
+    // dW[N][K] = dy^T . (q * absmax / 127) (zeros when M == 0)
+    if (N > 0 && M == 0) {
+        if (cudaMemsetAsync(dW, 0, 4 * static_cast<size_t>(N) * k, s) != cudaSuccess) return MMF_ERR_CUDA;
+    } else if (N > 0) {
+        CUtensorMap mb, mr;
+        if ((st = encode_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy, N, M, 2 * N, 64, kBwKs,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) != MMF_OK)
+            return st;
+        if ((st = encode_2d(&mr, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, M, K, kBwRows, kBwKs,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)) != MMF_OK)
+            return st;
+        BwParams bp{};
+        bp.out = dW;
+        bp.absmax = absmax;
+        bp.K = static_cast<int>(K);
+        bp.cols = static_cast<int>(N);
+        bp.contr = static_cast<int>(M);
+        bp.row_tiles = row_tiles;
+        bp.num_tiles = row_tiles * static_cast<int>((N + kBwCols - 1) / kBwCols);
+        const dim3 grid(static_cast<unsigned>(bp.num_tiles < dev->num_sms ? bp.num_tiles : dev->num_sms));
+        if ((st = launch(gemm_bwd_kernel<1>, grid, dim3(kBwThreads), BwLayout<1>::smem_bytes, s, false, mb, mr, bp)) !=
+            MMF_OK)
+            return st;
+    }
     if (M > 0 && (st = launch(rmsnorm_bwd_kernel, dim3(static_cast<unsigned>(M)), dim3(kBwdThreads), 0, s, false, x,
                               gamma, static_cast<const float*>(dr), scale, eps, static_cast<int>(K), dx, inv)) != MMF_OK)
         return st;
+    const auto blocks = [](int64_t count) { return dim3(static_cast<unsigned>((count + kBwdThreads - 1) / kBwdThreads)); };
     if (M > 0 && (st = launch(dgamma_partial_kernel, dim3(blocks(K).x, static_cast<unsigned>(chunks)), dim3(kBwdThreads),
                               0, s, false, x, static_cast<const float*>(dr), static_cast<const float*>(inv), M,
                               static_cast<int>(K), part)) != MMF_OK)

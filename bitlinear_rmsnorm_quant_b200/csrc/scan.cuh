@@ -23,16 +23,41 @@ namespace mmf {
 constexpr int kScanWarps = 32;
 
 // sigma(v) = 1 / (1 + e^-v) with the hardware exponential and reciprocal
-// (a few ulp: the recurrence is instruction-bound with the IEEE forms, and
-// its state is compared with the oracle to fp32-level tolerances anyway).
-__device__ __forceinline__ float sigmoid_f(float v) { return __fdividef(1.0f, 1.0f + __expf(-v)); }
+// (a few ulp: the recurrence is bound by the transcendental pipe with the
+// IEEE forms, and its state is compared with the oracle to fp32-level
+// tolerances anyway).  The sigmoids of one token share one reciprocal:
+// with d_i = 1 + e^-v_i, 1 / (d_1 d_2) gives sigma(v_1) = d_2 / (d_1 d_2)
+// and sigma(v_2) = d_1 / (d_1 d_2) (three of the pipe's operations instead of
+// four; five instead of six for three sigmoids).  Inputs are clamped below at
+// -28 so that a product of three d stays finite (e^28 < 1.5e12); sigma(-28)
+// is 7e-13, so the clamp changes a gate by less than that.
+constexpr float kScanClamp = -28.0f;
+
+__device__ __forceinline__ float sig_den(float v) { return 1.0f + __expf(-fmaxf(v, kScanClamp)); }
+
+__device__ __forceinline__ void sigmoid2(float a, float b, float& sa, float& sb) {
+    const float da = sig_den(a), db = sig_den(b);
+    const float r = __fdividef(1.0f, da * db);
+    sa = r * db;
+    sb = r * da;
+}
+
+__device__ __forceinline__ void sigmoid3(float a, float b, float c, float& sa, float& sb, float& sc) {
+    const float da = sig_den(a), db = sig_den(b), dc = sig_den(c);
+    const float dab = da * db;
+    const float r = __fdividef(1.0f, dab * dc);
+    const float rc = r * dc;  // 1 / (da db)
+    sa = rc * db;
+    sb = rc * da;
+    sc = r * dab;
+}
 
 __device__ __forceinline__ void bf16x2_to_f(uint32_t w, float& lo, float& hi) {
     lo = __uint_as_float(w << 16);
     hi = __uint_as_float(w & 0xFFFF0000u);
 }
 
-__global__ void __launch_bounds__(kScanWarps * 32) mlgru_scan_kernel(const uint16_t* __restrict__ f_pre,
+__global__ void __launch_bounds__(kScanWarps * 32, 1) mlgru_scan_kernel(const uint16_t* __restrict__ f_pre,
                                                                      const uint16_t* __restrict__ c_pre,
                                                                      const uint16_t* __restrict__ g_pre,
                                                                      const float* __restrict__ h0, int T, int D,
@@ -55,8 +80,10 @@ __global__ void __launch_bounds__(kScanWarps * 32) mlgru_scan_kernel(const uint1
             float fp0, fp1, cp0, cp1;
             bf16x2_to_f(__ldg(reinterpret_cast<const uint32_t*>(f_pre + idx(t))), fp0, fp1);
             bf16x2_to_f(__ldg(reinterpret_cast<const uint32_t*>(c_pre + idx(t))), cp0, cp1);
-            const float f0 = sigmoid_f(fp0), f1 = sigmoid_f(fp1);
-            const float c0 = __fmul_rn(cp0, sigmoid_f(cp0)), c1 = __fmul_rn(cp1, sigmoid_f(cp1));
+            float f0, f1, sc0, sc1;
+            sigmoid2(fp0, cp0, f0, sc0);
+            sigmoid2(fp1, cp1, f1, sc1);
+            const float c0 = __fmul_rn(cp0, sc0), c1 = __fmul_rn(cp1, sc1);
             b0 = __fadd_rn(__fmul_rn(f0, b0), __fmul_rn(__fsub_rn(1.0f, f0), c0));
             b1 = __fadd_rn(__fmul_rn(f1, b1), __fmul_rn(__fsub_rn(1.0f, f1), c1));
             a0 = __fmul_rn(a0, f0);
@@ -87,12 +114,13 @@ __global__ void __launch_bounds__(kScanWarps * 32) mlgru_scan_kernel(const uint1
             bf16x2_to_f(__ldg(reinterpret_cast<const uint32_t*>(f_pre + idx(t))), fp0, fp1);
             bf16x2_to_f(__ldg(reinterpret_cast<const uint32_t*>(c_pre + idx(t))), cp0, cp1);
             bf16x2_to_f(__ldg(reinterpret_cast<const uint32_t*>(g_pre + idx(t))), gp0, gp1);
-            const float f0 = sigmoid_f(fp0), f1 = sigmoid_f(fp1);
-            const float c0 = __fmul_rn(cp0, sigmoid_f(cp0)), c1 = __fmul_rn(cp1, sigmoid_f(cp1));
+            float f0, f1, sc0, sc1, g0, g1;
+            sigmoid3(fp0, cp0, gp0, f0, sc0, g0);
+            sigmoid3(fp1, cp1, gp1, f1, sc1, g1);
+            const float c0 = __fmul_rn(cp0, sc0), c1 = __fmul_rn(cp1, sc1);
             h0v = __fadd_rn(__fmul_rn(f0, h0v), __fmul_rn(__fsub_rn(1.0f, f0), c0));
             h1v = __fadd_rn(__fmul_rn(f1, h1v), __fmul_rn(__fsub_rn(1.0f, f1), c1));
-            const __nv_bfloat162 ov =
-                __floats2bfloat162_rn(__fmul_rn(sigmoid_f(gp0), h0v), __fmul_rn(sigmoid_f(gp1), h1v));
+            const __nv_bfloat162 ov = __floats2bfloat162_rn(__fmul_rn(g0, h0v), __fmul_rn(g1, h1v));
             *reinterpret_cast<__nv_bfloat162*>(o + idx(t)) = ov;
         }
         // the state after the last token: the warp whose chunk ends at T (warp 0 when T == 0)

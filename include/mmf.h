@@ -195,11 +195,16 @@ int mmf_mlgru_scan(const uint16_t* f_pre, const uint16_t* c_pre,
  *   dgamma = sum over tokens of dr * x * inv,  inv = 1 / sqrt(sum x^2 / K + eps).
  * dy: bf16 [M][N]; x, gamma, eps, packed, scale as for the forward;
  * dx: bf16 [M][K]; dgamma: fp32 [K]; dW: fp32 [N][K] (the latent weights'
- * gradient); all overwritten.  The two products are bf16 GEMMs with fp32
- * accumulation (cuBLAS, opened on the first call; MMF_ERR_CUDA if it cannot
- * be loaded); dy * absmax / 127 is rounded to bf16 for dW.  workspace: at
- * least mmf_bwd_workspace_bytes(M, K, N) bytes, no initialisation needed.
- * Sizes as the forward, with M * N and M * K below 2^31 and M <= 4194240.
+ * gradient); all overwritten.  The two products run on the tensor cores in
+ * this library's own kernel (bf16 operands, fp32 accumulation): for dr the
+ * ternary weights are unpacked from the 2-bit codes (exact), for dW each
+ * token's codes are scaled by absmax / 127 and rounded to bf16 as they are
+ * loaded.  An empty contraction gives zeros (M == 0: dW = 0, dgamma = 0;
+ * N == 0: dx = 0).  workspace: at least mmf_bwd_workspace_bytes(M, K, N)
+ * bytes, no initialisation needed.  Sizes as the forward, with N a multiple
+ * of 8 (dy rows are read by TMA) and M <= 4194240; buffers of an empty extent
+ * (x, dx and workspace when M == 0; dW when N == 0; dy and packed when either
+ * is 0) may be NULL.
  */
 size_t mmf_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N);
 int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma,

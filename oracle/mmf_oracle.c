@@ -171,11 +171,11 @@ void orc_rmsnorm_quant(const uint16_t* x, const float* gamma, float eps,
 void orc_ternary_acc(const int8_t* q, const int8_t* wt, int64_t M, int64_t K,
                      int64_t N, int32_t* acc) {
 #ifdef _OPENMP
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for collapse(2) schedule(static)
 #endif
     for (int64_t m = 0; m < M; ++m) {
-        const int8_t* qm = q + m * K;
         for (int64_t n = 0; n < N; ++n) {
+            const int8_t* qm = q + m * K;
             const int8_t* wn = wt + n * K;
             int32_t s = 0;
             for (int64_t k = 0; k < K; ++k) {

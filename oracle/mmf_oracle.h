@@ -28,9 +28,9 @@
  *
  * Error behaviour: none of these functions checks its arguments; the caller
  * passes valid buffers of the sizes above.  The functions are sequential except
- * orc_ternary_acc, whose outer loop over tokens may run on OpenMP threads (the
- * result does not depend on the thread count: every acc element is a plain
- * integer sum formed by one thread).
+ * orc_ternary_acc, whose (token, output row) pairs may be shared out among
+ * OpenMP threads (the result does not depend on the thread count: every acc
+ * element is a plain integer sum formed by one thread).
  */
 #ifndef MMF_ORACLE_H
 #define MMF_ORACLE_H

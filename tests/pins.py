@@ -331,10 +331,15 @@ def check_glu_gate(orc):
     ref = gv * expit(gv) * uv
     # one bf16 rounding (2^-8 relative) plus the fp32 steps before it
     assert (np.abs(p - ref) <= np.abs(ref) * (2.0 ** -8 + 2.0 ** -20) + 1e-30).all()
-    # SiLU(0) = 0 and u = 0 give exact zeros
-    z = np.zeros(4, dtype=np.uint16)
-    assert (orc.glu_gate(z, u[:4]) == 0).all() or (_bf16_bits_to_f64(orc.glu_gate(z, u[:4])) == 0).all()
-    assert (_bf16_bits_to_f64(orc.glu_gate(g[:64], np.zeros(64, dtype=np.uint16))) == 0).all()
+    # SiLU(0) = +0 * sigma(0) = +0, and +0 * u is a zero carrying the sign of u
+    # (IEEE product sign rule): the exact bit pattern, not only the value
+    z = np.zeros(64, dtype=np.uint16)
+    want = np.where(np.signbit(_bf16_bits_to_f64(u[:64])), 0x8000, 0x0000).astype(np.uint16)
+    assert np.array_equal(orc.glu_gate(z, u[:64]), want)
+    # u = +0 gives a zero of g's sign (SiLU(g) has the sign of g)
+    pz = orc.glu_gate(g[:64], np.zeros(64, dtype=np.uint16))
+    assert (_bf16_bits_to_f64(pz) == 0).all()
+    assert np.array_equal(np.signbit(_bf16_bits_to_f64(pz)), np.signbit(_bf16_bits_to_f64(g[:64])))
     # SiLU(v) - SiLU(-v) = v, with u = 1: within two bf16 roundings
     one = _bits_of(np.ones(256, dtype=np.float32))
     gp = _bits_of(np.linspace(-8, 8, 256).astype(np.float32).astype(np.float64).astype(np.float32)

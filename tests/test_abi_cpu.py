@@ -46,9 +46,11 @@ def test_library_is_sm100a_only():
 def test_sizes(L):
     assert L.mmf_packed_bytes(2560, 6912) == 2560 * 6912 // 4
     assert L.mmf_packed_bytes(-1, 128) == 0
-    # small M takes the fused decode kernel: no workspace
+    # one token takes the fused decode kernel: no workspace
     assert L.mmf_workspace_bytes(1, 2560, 2560) == 0
-    assert L.mmf_workspace_bytes(8, 6912, 2560) == 0
+    # 2 .. 32 tokens: the codes in the decode tensor-core kernel's operand layout
+    # (16 or 32 token rows per 128-wide K chunk) + absmax + qsum, 256-byte aligned
+    assert L.mmf_workspace_bytes(8, 6912, 2560) == 16 * 6912 + 2 * 256
     # large M: int8 codes + absmax + qsum, each 256-byte aligned
     M, K = 8192, 2048
     assert L.mmf_workspace_bytes(M, K, 5632) == M * K + 2 * ((4 * M + 255) // 256 * 256)
@@ -181,12 +183,18 @@ def test_shape_limits(L):
 
 
 def test_workspace_sizes_follow_the_path(L):
-    # the decode path (up to 8 tokens whose activations fit in shared memory) needs none;
-    # the large-M path needs the codes, the per-token absmax and code sums
+    # one token (the CUDA-core decode kernel) needs none; 2 .. 32 tokens (the
+    # decode tensor-core kernel) need the codes as 16 or 32 operand rows per K
+    # chunk and the per-token absmax and code sums; the large-M path the codes,
+    # absmax and sums of every token
+    a256 = lambda v: (v + 255) // 256 * 256
     for K in (128, 2560, 6912):
         assert L.mmf_workspace_bytes(1, K, 256) == 0
-        assert L.mmf_workspace_bytes(8, K, 256) == 0
-        assert L.mmf_workspace_bytes(9, K, 256) >= 9 * K + 8 * 9
+        for M in (2, 8, 16):
+            assert L.mmf_workspace_bytes(M, K, 256) == a256(16 * K) + 2 * a256(4 * M)
+        for M in (17, 32):
+            assert L.mmf_workspace_bytes(M, K, 256) == a256(32 * K) + 2 * a256(4 * M)
+        assert L.mmf_workspace_bytes(33, K, 256) == a256(33 * K) + 2 * a256(4 * 33)
         assert L.mmf_workspace_bytes(8192, K, 256) >= 8192 * K + 8 * 8192
     # a single token too wide for the decode kernel's shared memory takes the large-M path
     assert L.mmf_workspace_bytes(1, 65536, 256) >= 65536

@@ -38,7 +38,19 @@ def test_reference_arm_prints_the_contract_line():
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
 
 
-@pytest.mark.parametrize("workload", ["smoke-256", "decode-2.7b-m1"])
+def test_reference_arm_default_workload_states_host_cores():
+    """The default workload (the training-batch forward) on the reference arm:
+    the oracle on a token sample, the threads it used and the host's cores."""
+    r = _run("--impl", "reference", "--steps", "2", "--warmup", "3")
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads([ln for ln in r.stdout.splitlines() if ln.strip().startswith("{")][0])
+    assert d["config"]["workload"] == "train-fwd-1.3b" and d["config"]["M"] == 524288
+    cb = d["cpu_baseline"]
+    assert cb["host_cores"] >= 1 and cb["threads"] >= 1 and cb["cores"] == cb["threads"]
+    assert "extrapolated" in cb["sample"]
+
+
+@pytest.mark.parametrize("workload", ["smoke-256", "decode-2.7b-m1", "train-fwd-1.3b"])
 def test_our_arm_fails_loudly_without_a_device(workload):
     r = _run("--workload", workload, "--steps", "3", "--warmup", "3", "--no-cpu-baseline")
     assert r.returncode != 0

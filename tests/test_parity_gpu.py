@@ -82,11 +82,14 @@ def test_pack_special_matrices(oracle):
 
 @pytest.mark.parametrize("M,K,outliers", [(16, 256, 0.0), (5, 128, 0.0), (300, 2048, 0.0), (37, 6912, 0.01),
                                           (64, 5632, 0.0),
-                                          # large M: the persistent streaming quantiser
-                                          (4100, 1024, 0.0), (4096, 7168, 0.01), (5000, 128, 0.0),
-                                          (4097, 7296, 0.0),
-                                          # one row buffer per warp up to its largest K; beyond it, a CTA per row
-                                          (4096, 11264, 0.0), (4096, 11392, 0.01)])
+                                          # large M: the persistent register kernel, one to four warps per
+                                          # row (K <= 2048, 4096, 6144, 8192), ragged lanes at each width
+                                          (4100, 1024, 0.0), (5000, 128, 0.0), (4096, 2048, 0.01),
+                                          (4099, 2560, 0.01), (4096, 4096, 0.0), (4097, 5632, 0.0),
+                                          (4096, 6144, 0.01), (4096, 6912, 0.01), (4096, 7168, 0.01),
+                                          (4097, 7296, 0.0), (4096, 8192, 0.0),
+                                          # beyond its largest K, a CTA per row
+                                          (4096, 8320, 0.0), (4096, 11392, 0.01)])
 def test_quantize_act(oracle, M, K, outliers):
     x, g, _ = make_layer(9, M, K, 1, outlier_frac=outliers)
     q, a = mmf.quantize_act(x.to(DEV), g.to(DEV), EPS)
@@ -115,12 +118,15 @@ def test_quantize_special_rows(oracle):
 # -- ternary contraction: int32 bit-exact on the kernel's own q and packed W --------------
 
 ACC_SHAPES = [
-    # (M, K, N) decode GEMV path (M <= 8)
-    (1, 128, 1), (1, 256, 256), (2, 1024, 1000), (3, 2560, 333), (8, 6912, 2560), (5, 2816, 1024),
-    (1, 6912, 20000), (4, 4096, 9000),   # weight ring refilled many times per CTA
-    # tcgen05 path: several 128-row tiles, token tiles, K stages, ragged tails
-    (9, 256, 300), (16, 256, 256), (17, 384, 129), (32, 2560, 640), (100, 1024, 257), (256, 512, 384),
-    (300, 384, 300), (513, 2048, 200),
+    # (M, K, N) CUDA-core decode kernel (one token)
+    (1, 128, 1), (1, 256, 256), (1, 6912, 20000),   # weight ring refilled many times per CTA
+    # decode tensor-core kernel (2 .. 32 tokens): slabs of 8 .. 128 rows, ragged slabs, the code ring
+    # refilled (K = 6912: 54 chunks), 16 and 32 operand rows
+    (2, 1024, 1000), (3, 2560, 333), (8, 6912, 2560), (5, 2816, 1024), (4, 4096, 9000), (9, 256, 300),
+    (16, 256, 256), (17, 384, 129), (32, 2560, 640), (32, 6912, 700), (24, 2560, 13824), (2, 128, 8),
+    (31, 8192, 40000),
+    # large-M tcgen05 path: several 128-row tiles, token tiles, K stages, ragged tails
+    (33, 2048, 500), (100, 1024, 257), (256, 512, 384), (300, 384, 300), (513, 2048, 200),
 ]
 
 
@@ -255,6 +261,77 @@ def test_single_token_matches_large_m_path(oracle, case):
     assert y_rel_error(bits_np(y1), y_ref) <= Y_REL_TOL
 
 
+@pytest.mark.parametrize("M", [2, 3, 5, 8, 13, 16, 17, 24, 32])
+@pytest.mark.parametrize("K", [2560, 6912])
+def test_decode_codes_match_large_m_path(oracle, M, K):
+    """The decode tensor-core path (2 .. 32 tokens) keeps its codes in the MMA's
+    operand layout, with zero rows up to 16 or 32 tokens, and never hands them
+    out.  M tokens on it against the same tokens as the first rows of a
+    64-token batch (codes in row-major order, which the quantiser test compares
+    with the oracle, then the large-M tensor-core kernel): bit-equal y means
+    equal codes, sums and absmax (a code off by one changes acc for every
+    output row whose weight at that k is not 0).  Rows of the 2.7B decode
+    workload, 1% outlier channels x20."""
+    N = 512
+    wl = WL.decode_2p7b(8)
+    x, g, W = make_layer(wl.seed, 64, K, N, index=40 + M, outlier_frac=wl.outlier_frac)
+    x[0, :] = x[0, :] * 0.0 + 1.5          # a constant token (every |r| ties)
+    packed, scale = _pack(W)
+    xd, gd = x.to(DEV), g.to(DEV)
+    nt = 16 if M <= 16 else 32               # two different paths: operand layout vs row-major codes
+    assert mmf.workspace_bytes(M, K, N) < nt * K + 1024 < mmf.workspace_bytes(64, K, N)
+    y_small = mmf.bitlinear_fwd(xd[:M].contiguous(), gd, packed, scale, N, EPS)
+    y_big = mmf.bitlinear_fwd(xd, gd, packed, scale, N, EPS)
+    torch.cuda.synchronize()
+    assert torch.equal(y_small, y_big[:M])
+    y_ref, _ = oracle.bitlinear(bits_np(x[:M]), g.numpy(), EPS, W.numpy(), EPS_W)
+    assert y_rel_error(bits_np(y_small), y_ref) <= Y_REL_TOL
+
+
+def test_training_batch_forward_sampled(oracle):
+    """The training-batch forward's largest projection, 5632 -> 2048 at
+    M = 2^8 * 2048 = 524288 tokens (its codes take M*K = 2.95e9 bytes, past
+    2^31), full size on the GPU through the C ABI: the int8 codes and absmax of
+    64 sampled tokens (half of them beyond row 2^31 / K) against the oracle,
+    their int32 accumulators bit-exact on the kernel's own codes, and y within
+    the layer bar.  x is drawn on the device; the oracle reads the sampled
+    rows' bytes back from it."""
+    wl = WL.TRAIN_FWD_1P3B
+    p = [p for p in wl.projections if p.name == "down"][0]
+    M, K, N = wl.M, p.K, p.N
+    assert M * K > 2 ** 31
+    rng = np.random.default_rng(11)
+    edge = (2 ** 31) // K
+    rows = np.sort(np.concatenate([rng.choice(edge, 32, replace=False),
+                                   edge + rng.choice(M - edge, 31, replace=False), [M - 1]]))
+    xd = I.activations(wl.seed, M, K, index=p.input_index, device=DEV)
+    g = I.gamma(wl.seed, K, index=p.input_index)
+    W = I.latent_weights(wl.seed, N, K, index=6)
+    gd = g.to(DEV)
+    packed, scale = _pack(W)
+    ridx = torch.as_tensor(rows, device=DEV)
+    x_rows = bits_np(xd[ridx])
+    q, a = mmf.quantize_act(xd, gd, EPS)
+    q_rows, a_rows = q[ridx].cpu().numpy(), a[ridx].cpu().numpy()
+    acc = mmf.ternary_acc(q, packed, N)
+    acc_rows = acc[ridx].cpu().numpy()
+    del acc, q
+    y = mmf.bitlinear_fwd(xd, gd, packed, scale, N, EPS)
+    y_rows = bits_np(y[ridx])
+    torch.cuda.synchronize()
+    del y, xd
+    q_ref, a_ref = oracle.rmsnorm_quant(x_rows, g.numpy(), EPS)
+    frac, mx = q_diff_stats(q_rows, q_ref)
+    assert mx <= 1 and frac <= Q_MAX_DIFF_FRAC
+    assert np.allclose(a_rows, a_ref, rtol=2e-7, atol=0)
+    wt, bad = oracle.decode_packed(packed.cpu().numpy().view(np.uint32), K)
+    assert bad == 0
+    assert np.array_equal(acc_rows, oracle.ternary_acc(q_rows, wt))
+    y_ref, beta = oracle.bitlinear(x_rows, g.numpy(), EPS, W.numpy(), EPS_W)
+    assert np.float32(scale.item()) == beta
+    assert y_rel_error(y_rows, y_ref) <= Y_REL_TOL
+
+
 # -- GLU channel mixer: down projection with SiLU(g) * u fused in -----------------------------
 
 @pytest.mark.parametrize("M,K,N", [(1, 6912, 2560), (3, 2816, 1024), (8, 5632, 2048), (1, 128, 16),
@@ -338,8 +415,8 @@ def test_mlgru_scan_continues_across_calls():
 
 # -- backward with the straight-through estimator --------------------------------------------
 
-@pytest.mark.parametrize("M,K,N", [(1, 256, 128), (16, 512, 256), (64, 1024, 300), (300, 384, 1024),
-                                   (1000, 2048, 512)])
+@pytest.mark.parametrize("M,K,N", [(1, 256, 128), (16, 512, 256), (64, 1024, 296), (300, 384, 1024),
+                                   (1000, 2048, 512), (513, 256, 72), (257, 640, 1000)])
 def test_bwd_parity(oracle, M, K, N):
     x, g, W = make_layer(24, M, K, N)
     dy = I.activations(24, M, N, index=7)
@@ -348,14 +425,68 @@ def test_bwd_parity(oracle, M, K, N):
     torch.cuda.synchronize()
     wt, beta = oracle.absmean_ternary(W.numpy(), EPS_W)
     dx_ref, dg_ref, dW_ref = oracle.bitlinear_bwd(bits_np(dy), bits_np(x), g.numpy(), EPS, wt, beta)
-    # bf16 GEMM operands (dy * absmax / 127 rounded to bf16) and fp32 accumulation:
-    # errors well inside the layer's 1e-2 bar, relative to each output's scale
+    # tensor-core products with fp32 accumulation; x_q = q * absmax / 127 rounded
+    # to bf16 for dW: errors well inside the layer's 1e-2 bar, relative to each
+    # output's scale
     def rel(a, b):
         b = np.asarray(b, dtype=np.float64)
         return np.abs(np.asarray(a, dtype=np.float64) - b).max() / max(np.abs(b).max(), 1e-30)
     assert rel(bf16_to_f64(bits_np(dx.cpu())), bf16_to_f64(dx_ref)) <= 1e-2
     assert rel(dg.cpu().numpy(), dg_ref) <= 1e-3
     assert rel(dW.cpu().numpy(), dW_ref) <= 1e-2
+
+
+def test_bwd_dr_exact_on_exact_inputs(oracle):
+    """dy with few significant bits and ternary weights: every product and
+    partial sum of dr = dy . w~ is exact in fp32, so dx matches the oracle's
+    fp64 evaluation to its own bf16 rounding, whatever the order of the sums;
+    and dW of one token is dy^T times the token's bf16 x_q exactly."""
+    M, K, N = 1, 256, 192
+    rng = np.random.default_rng(3)
+    x, g, W = make_layer(25, M, K, N)
+    dy = torch.from_numpy(rng.integers(-8, 9, size=(M, N)).astype(np.float32)).to(torch.bfloat16)
+    packed, scale = _pack(W)
+    dx, dg, dW = mmf.bitlinear_bwd(dy.to(DEV), x.to(DEV), g.to(DEV), packed, scale, EPS)
+    torch.cuda.synchronize()
+    wt, beta = oracle.absmean_ternary(W.numpy(), EPS_W)
+    dx_ref, dg_ref, dW_ref = oracle.bitlinear_bwd(bits_np(dy), bits_np(x), g.numpy(), EPS, wt, beta)
+    # dW[n][k] = dy[n] * bf16(q[k] * a / 127): one bf16 rounding of x_q, then an exact product
+    q, a = oracle.rmsnorm_quant(bits_np(x), g.numpy(), EPS)
+    xq = (q[0].astype(np.float32) * (np.float32(a[0]) / np.float32(127.0))).astype(np.float32)
+    xq_b = bf16_to_f64(bits_np(torch.from_numpy(xq).to(torch.bfloat16)))
+    assert np.array_equal(dW.cpu().numpy().astype(np.float64), np.outer(dy.float().numpy()[0], xq_b))
+    # dx: exact dr, then the RMSNorm backward in fp64 (sums in another order): one bf16 step at most
+    dxv, dxr = bf16_to_f64(bits_np(dx.cpu())), bf16_to_f64(dx_ref)
+    assert (np.abs(dxv - dxr) <= np.abs(dxr) * 2.0 ** -8 + 1e-30).all()
+    assert np.abs(dg.cpu().numpy() - dg_ref).max() <= 1e-5 * np.abs(dg_ref).max()
+
+
+@pytest.mark.parametrize("M,N", [(0, 64), (16, 0)])
+def test_bwd_empty_contractions(oracle, M, N):
+    """An empty contraction gives zero products: M = 0 (no tokens) gives dW = 0
+    and dgamma = 0; N = 0 (no outputs) gives dr = 0, so dx = 0."""
+    K = 256
+    x = torch.randn(M, K).to(torch.bfloat16).to(DEV)
+    g = torch.ones(K, device=DEV)
+    packed, scale = mmf.pack_ternary(torch.randn(max(N, 1), K, device=DEV))
+    dy = torch.randn(M, N).to(torch.bfloat16).to(DEV)
+    dx, dg, dW = mmf.bitlinear_bwd(dy, x, g, packed[:N] if N else packed[:0], scale, EPS)
+    torch.cuda.synchronize()
+    assert dW.shape == (N, K) and (dW == 0).all()
+    assert (dg == 0).all()
+    if M:
+        assert (dx.float() == 0).all()
+
+
+def test_bwd_rejects_unaligned_output_width():
+    """dy rows are read by TMA: N must be a multiple of 8 (16-byte row pitch)."""
+    L = mmf.lib()
+    K, M, N = 256, 4, 300
+    buf = torch.zeros(1 << 20, dtype=torch.uint8, device=DEV)
+    p = buf.data_ptr()
+    assert L.mmf_bitlinear_bwd(p, p, p, 1e-6, p, p, M, K, N, p, p, p, p, buf.numel(),
+                               torch.cuda.current_stream().cuda_stream) == 2   # MMF_ERR_UNSUPPORTED_SHAPE
+    mmf.check_async()
 
 
 def test_empty_problems():

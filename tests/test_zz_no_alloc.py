@@ -28,7 +28,9 @@ def _noalloc(x, g, packed, scale, N, y):
                                                torch.cuda.current_stream().cuda_stream)
 
 
-@pytest.mark.parametrize("M,K,N", [(1000, 2048, 512), (300, 384, 300), (4, 2560, 1000)])
+# (4096, 2048, 512): the persistent streaming quantiser and the 256-token
+# tensor-core tile write and read the static scratch
+@pytest.mark.parametrize("M,K,N", [(1000, 2048, 512), (300, 384, 300), (4, 2560, 1000), (4096, 2048, 512)])
 def test_noalloc_matches_workspace_forward_twice(M, K, N):
     from bitlinear_rmsnorm_quant_b200 import build
     build.build()
