@@ -507,7 +507,7 @@ class Step:
                                    self.packed[l, j].data_ptr(), self.scales[l, j].data_ptr(), Mc, p.K, p.N,
                                    y[j].data_ptr(), self.ws.data_ptr(), self.ws.numel(), self.flags)))
                     if count:
-                        self.launches_per_step += 1 if mmf.workspace_bytes(Mc, p.K, p.N) == 0 else 2
+                        self.launches_per_step += mmf.fwd_launches(Mc, p.K, p.N)
                         self.bytes_per_step += p.N * p.K // 4 + 2 * Mc * p.N + 4 + 2 * (2 * Mc * K) + 4 * K
                         self.ops_per_step += proj_ops(Mc, p.K, p.N)
                     continue
@@ -519,8 +519,8 @@ class Step:
                                   (x.data_ptr(), g.data_ptr(), wl.eps, Mc, K, arr, len(js), self.ws.data_ptr(),
                                    self.ws.numel(), self.flags)))
                     if count:
-                        tc = mmf.workspace_bytes(Mc, K, 1) > 0
-                        self.launches_per_step += (1 + len(js)) if tc else 1
+                        self.launches_per_step += mmf.fwd_launches(Mc, K, sum(wl.projections[j].N for j in js),
+                                                                   len(js))
                 else:
                     for j in js:
                         p = wl.projections[j]
@@ -529,7 +529,7 @@ class Step:
                                        self.scales[l, j].data_ptr(), Mc, p.K, p.N, y[j].data_ptr(),
                                        self.ws.data_ptr(), self.ws.numel())))
                         if count:
-                            self.launches_per_step += 1 if mmf.workspace_bytes(Mc, p.K, p.N) == 0 else 2
+                            self.launches_per_step += mmf.fwd_launches(Mc, p.K, p.N)
                 if count:
                     for j in js:
                         p = wl.projections[j]

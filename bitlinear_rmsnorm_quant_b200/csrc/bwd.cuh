@@ -93,4 +93,124 @@ __global__ void __launch_bounds__(kBwdThreads) dgamma_final_kernel(const double*
     dgamma[k] = static_cast<float>(s * static_cast<double>(__ldg(beta)));
 }
 
+// RMSNorm backward and the dgamma partial sums in one pass over HBM (K <=
+// 8192): a CTA takes kBwdFusedRows consecutive token rows; thread t owns the
+// 8-column chunks c = t + 256 i (i < CPT) and keeps its columns' dgamma
+// partial sums (fp64) in registers over the CTA's rows.  Per row it reads x
+// and dr (16- and 32-byte loads, kept in L1), forms the row's fp64 sums of
+// x^2 and gamma beta dr x (a warp tree, then the warps in index order), then
+// reads the same lines again from L1 to write dx and add dr x inv to its
+// partials, rows in order.  The CTA's partials go to part[blockIdx.x][k];
+// dgamma_final_kernel sums them over the CTAs in order.
+constexpr int kBwdFusedRows = 16;
+constexpr int kBwdFusedMaxK = kBwdThreads * 8 * 4;
+
+__device__ __forceinline__ void load_x8_dr8(const uint16_t* x, const float* dr, int64_t off, float (&xv)[8],
+                                            float (&dv)[8]) {
+    const uint4 xw = __ldg(reinterpret_cast<const uint4*>(x + off));
+    const float4 da = __ldg(reinterpret_cast<const float4*>(dr + off));
+    const float4 db = __ldg(reinterpret_cast<const float4*>(dr + off) + 1);
+    const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        xv[2 * e] = __uint_as_float(w[e] << 16);
+        xv[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+    dv[0] = da.x; dv[1] = da.y; dv[2] = da.z; dv[3] = da.w;
+    dv[4] = db.x; dv[5] = db.y; dv[6] = db.z; dv[7] = db.w;
+}
+
+template <int CPT>
+__global__ void __launch_bounds__(kBwdThreads) rmsnorm_bwd_fused_kernel(const uint16_t* __restrict__ x,
+                                                                        const float* __restrict__ gamma,
+                                                                        const float* __restrict__ dr,
+                                                                        const float* __restrict__ beta, float eps,
+                                                                        int K, int64_t M,
+                                                                        uint16_t* __restrict__ dx,
+                                                                        double* __restrict__ part) {
+    __shared__ double red_s[2][kBwdThreads / 32], red_d[2][kBwdThreads / 32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int C = K >> 3;
+    const double bt = static_cast<double>(__ldg(beta));
+    const float4* g4 = reinterpret_cast<const float4*>(gamma);
+    double acc[CPT][8];
+#pragma unroll
+    for (int i = 0; i < CPT; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[i][e] = 0.0;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBwdFusedRows;
+    const int64_t m1 = m0 + kBwdFusedRows < M ? m0 + kBwdFusedRows : M;
+    for (int64_t m = m0; m < m1; ++m) {
+        const int buf = static_cast<int>(m - m0) & 1;
+        const int64_t row = m * static_cast<int64_t>(K);
+        double s2 = 0.0, dot = 0.0;
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = threadIdx.x + kBwdThreads * i;
+            if (c < C) {
+                float xv[8], dv[8];
+                load_x8_dr8(x, dr, row + 8 * c, xv, dv);
+                const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
+                const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const double xd = xv[e];
+                    s2 += xd * xd;
+                    dot += static_cast<double>(g[e]) * (bt * static_cast<double>(dv[e])) * xd;
+                }
+            }
+        }
+        s2 = warp_sum_f64(s2);
+        dot = warp_sum_f64(dot);
+        if (lane == 0) {
+            red_s[buf][warp] = s2;
+            red_d[buf][warp] = dot;
+        }
+        __syncthreads();  // (the other buffer was last read before the previous row's barrier)
+        s2 = 0.0;
+        dot = 0.0;
+#pragma unroll
+        for (int w = 0; w < kBwdThreads / 32; ++w) {
+            s2 += red_s[buf][w];
+            dot += red_d[buf][w];
+        }
+        const double inv = 1.0 / sqrt(s2 / static_cast<double>(K) + static_cast<double>(eps));
+        const double c2 = inv * inv * inv * dot / static_cast<double>(K);
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = threadIdx.x + kBwdThreads * i;
+            if (c < C) {
+                float xv[8], dv[8];
+                load_x8_dr8(x, dr, row + 8 * c, xv, dv);
+                const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
+                const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    uint32_t h[2];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int k = 2 * e + j;
+                        const double xd = xv[k], drd = static_cast<double>(dv[k]);
+                        const double gr = inv * static_cast<double>(g[k]) * (bt * drd) - xd * c2;
+                        h[j] = __bfloat16_as_ushort(__double2bfloat16(gr));
+                        acc[i][k] += drd * xd * inv;
+                    }
+                    o[e] = h[0] | (h[1] << 16);
+                }
+                *reinterpret_cast<uint4*>(dx + row + 8 * c) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = threadIdx.x + kBwdThreads * i;
+        if (c < C) {
+            double* pr = part + static_cast<int64_t>(blockIdx.x) * K + 8 * c;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pr[e] = acc[i][e];
+        }
+    }
+}
+
 }  // namespace mmf

@@ -1,4 +1,4 @@
-// gemv_tc.cuh -- decode-regime contraction for a few tokens (2 <= M <= 32) on
+// gemv_tc.cuh -- decode-regime contraction for a few tokens (9 <= M <= 32) on
 // the 5th-generation tensor cores.
 //
 // With M tokens the add/sub contraction on CUDA cores costs about M/4 integer

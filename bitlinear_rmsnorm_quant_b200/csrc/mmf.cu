@@ -139,9 +139,11 @@ mmf_status check_shape(int64_t M, int64_t K, int64_t N) {
 }
 
 // Small M: up to kDecodeTcMinM - 1 tokens the CUDA-core decode kernel (its
-// add/sub cost grows with M); from there to kDecodeTcMaxM the decode
-// tensor-core kernel after a quantiser launch; beyond, the large-M path.
-constexpr int64_t kDecodeTcMinM = 2;
+// add/sub cost grows with M, about M/4 integer instructions per weight); from
+// there to kDecodeTcMaxM the decode tensor-core kernel after a quantiser
+// launch (its cost is set by issuing K/32 MMAs per 128-row tile from one
+// thread, whatever M is); beyond, the large-M path.
+constexpr int64_t kDecodeTcMinM = 9;
 constexpr int64_t kDecodeTcMaxM = 32;
 
 bool takes_gemv(int64_t M, int64_t K) {
@@ -354,7 +356,7 @@ mmf_status fwd_impl(const uint16_t* x, const float* gamma, float eps, int64_t M,
     for (int i = 0; i < count; ++i) R += proj[i].N;
     if (R == 0) return MMF_OK;
     GemvPlan plan;
-    if (gemv_plan(static_cast<int>(M), static_cast<int>(K), R, dev->num_sms, &plan)) {
+    if (M < kDecodeTcMinM && gemv_plan(static_cast<int>(M), static_cast<int>(K), R, dev->num_sms, &plan)) {
         GemvParams p{};
         p.x = x;
         p.u = u;
@@ -459,6 +461,13 @@ size_t mmf_workspace_bytes(int64_t M, int64_t K, int64_t N) {
     return workspace_size_tc(M, K);
 }
 
+int mmf_fwd_launches(int64_t M, int64_t K, int64_t N, int count) {
+    if (check_shape(M, K, N) != MMF_OK || M == 0 || N == 0 || count < 1 || count > MMF_MAX_GROUP) return 0;
+    if (takes_gemv(M, K)) return 1;
+    if (takes_decode_tc(M, K)) return 2;
+    return 1 + count;
+}
+
 int mmf_pack_ternary(const float* W, int64_t N, int64_t K, float eps_w, uint32_t* packed, float* scale,
                      void* stream) {
     if (!(eps_w >= 0.0f) || eps_w > 1e30f) return MMF_ERR_INVALID_ARG;
@@ -513,7 +522,7 @@ int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t 
     if ((st = device_state(&dev)) != MMF_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     GemvPlan plan;
-    if (gemv_plan(static_cast<int>(M), static_cast<int>(K), N, dev->num_sms, &plan)) {
+    if (M < kDecodeTcMinM && gemv_plan(static_cast<int>(M), static_cast<int>(K), N, dev->num_sms, &plan)) {
         GemvParams p{};
         p.q_in = q;
         p.packed[0] = packed;
@@ -587,10 +596,14 @@ int mmf_bitlinear_fwd(const uint16_t* x, const float* gamma, float eps, const ui
     return fwd_impl(x, gamma, eps, M, K, &pr, 1, workspace, 0u, static_cast<cudaStream_t>(stream), dev);
 }
 
+// Rows summed per dgamma partial: the fused RMSNorm backward's CTA rows when
+// K allows it, else the two-stage column sum's chunk.
+int64_t bwd_partial_rows(int64_t K) { return K <= kBwdFusedMaxK ? kBwdFusedRows : kDgammaRows; }
+
 size_t mmf_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N) {
     if (check_shape(M, K, N) != MMF_OK) return 0;
     const size_t m = static_cast<size_t>(M), k = static_cast<size_t>(K);
-    const size_t chunks = (m + kDgammaRows - 1) / kDgammaRows;
+    const size_t chunks = (m + bwd_partial_rows(K) - 1) / bwd_partial_rows(K);
     // q, absmax, qsum, inv, dr (fp32), dgamma partials (fp64)
     return align256(m * k) + 3 * align256(4 * m) + align256(4 * m * k) + align256(8 * chunks * k);
 }
@@ -601,8 +614,9 @@ int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma,
     if (!(eps >= 0.0f) || eps > 1e30f) return MMF_ERR_INVALID_ARG;
     mmf_status st = check_shape(M, K, N);
     if (st != MMF_OK) return st;
-    // dy rows are read by TMA (row pitch a multiple of 16 bytes); the dgamma row chunks on grid.y
-    if ((N % 8) != 0 || M > 65535L * kDgammaRows) return MMF_ERR_UNSUPPORTED_SHAPE;
+    // dy rows are read by TMA (row pitch a multiple of 16 bytes); beyond the fused
+    // RMSNorm backward's K the dgamma row chunks go on grid.y
+    if ((N % 8) != 0 || (K > kBwdFusedMaxK && M > 65535L * kDgammaRows)) return MMF_ERR_UNSUPPORTED_SHAPE;
     if (M == 0 && N == 0) return MMF_OK;
     // buffers of an empty extent may be NULL
     if (!gamma || !scale || !dgamma) return MMF_ERR_INVALID_ARG;
@@ -630,7 +644,7 @@ int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma,
     float* dr = reinterpret_cast<float*>(b);
     b += align256(4 * m * k);
     double* part = reinterpret_cast<double*>(b);
-    const int chunks = static_cast<int>((M + kDgammaRows - 1) / kDgammaRows);
+    const int chunks = static_cast<int>((M + bwd_partial_rows(K) - 1) / bwd_partial_rows(K));
     const int row_tiles = static_cast<int>(K / kBwRows);
 
     if (M > 0 && (st = launch_quant(x, gamma, eps, M, K, q, absmax, qsum, s, false, dev->num_sms)) != MMF_OK) return st;
@@ -681,14 +695,27 @@ int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma,
             MMF_OK)
             return st;
     }
-    if (M > 0 && (st = launch(rmsnorm_bwd_kernel, dim3(static_cast<unsigned>(M)), dim3(kBwdThreads), 0, s, false, x,
-                              gamma, static_cast<const float*>(dr), scale, eps, static_cast<int>(K), dx, inv)) != MMF_OK)
-        return st;
     const auto blocks = [](int64_t count) { return dim3(static_cast<unsigned>((count + kBwdThreads - 1) / kBwdThreads)); };
-    if (M > 0 && (st = launch(dgamma_partial_kernel, dim3(blocks(K).x, static_cast<unsigned>(chunks)), dim3(kBwdThreads),
-                              0, s, false, x, static_cast<const float*>(dr), static_cast<const float*>(inv), M,
-                              static_cast<int>(K), part)) != MMF_OK)
-        return st;
+    if (M > 0 && K <= kBwdFusedMaxK) {
+        // dx and the dgamma partials in one pass over x and dr
+        const int cpt = static_cast<int>((K / 8 + kBwdThreads - 1) / kBwdThreads);  // 1, 2, 3 or 4
+        void (*kern)(const uint16_t*, const float*, const float*, const float*, float, int, int64_t, uint16_t*,
+                     double*) = cpt == 1   ? rmsnorm_bwd_fused_kernel<1>
+                                : cpt == 2 ? rmsnorm_bwd_fused_kernel<2>
+                                : cpt == 3 ? rmsnorm_bwd_fused_kernel<3>
+                                           : rmsnorm_bwd_fused_kernel<4>;
+        if ((st = launch(kern, dim3(static_cast<unsigned>(chunks)), dim3(kBwdThreads), 0, s, false, x, gamma,
+                         static_cast<const float*>(dr), scale, eps, static_cast<int>(K), M, dx, part)) != MMF_OK)
+            return st;
+    } else if (M > 0) {
+        if ((st = launch(rmsnorm_bwd_kernel, dim3(static_cast<unsigned>(M)), dim3(kBwdThreads), 0, s, false, x, gamma,
+                         static_cast<const float*>(dr), scale, eps, static_cast<int>(K), dx, inv)) != MMF_OK)
+            return st;
+        if ((st = launch(dgamma_partial_kernel, dim3(blocks(K).x, static_cast<unsigned>(chunks)), dim3(kBwdThreads), 0,
+                         s, false, x, static_cast<const float*>(dr), static_cast<const float*>(inv), M,
+                         static_cast<int>(K), part)) != MMF_OK)
+            return st;
+    }
     return launch(dgamma_final_kernel, blocks(K), dim3(kBwdThreads), 0, s, false, static_cast<const double*>(part), chunks,
                   static_cast<int>(K), scale, dgamma);
 }

@@ -36,6 +36,7 @@ SIGNATURES = {
     "mmf_version": (C.c_char_p, []),
     "mmf_packed_bytes": (_SZ, [_I64, _I64]),
     "mmf_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "mmf_fwd_launches": (_INT, [_I64, _I64, _I64, _INT]),
     "mmf_pack_ternary": (_INT, [_P, _I64, _I64, _F, _P, _P, _P]),
     "mmf_quantize_act": (_INT, [_P, _P, _F, _I64, _I64, _P, _P, _P]),
     "mmf_ternary_acc": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
@@ -115,6 +116,10 @@ def packed_bytes(N: int, K: int) -> int:
 
 def workspace_bytes(M: int, K: int, N: int) -> int:
     return int(lib().mmf_workspace_bytes(M, K, N))
+
+
+def fwd_launches(M: int, K: int, N: int, count: int = 1) -> int:
+    return int(lib().mmf_fwd_launches(M, K, N, count))
 
 
 def version() -> str:

@@ -68,12 +68,22 @@ const char* mmf_status_string(int status);
 /* Library version string, e.g. "mmf 0.1.0 sm_100a". */
 const char* mmf_version(void);
 
+/* Number of kernel launches one mmf_bitlinear_fwd_group call with `count`
+ * non-empty projections of N rows in total issues for this (M, K): 1 on the
+ * one-token decode path, 2 (quantiser + contraction) for 2 .. 32 tokens,
+ * 1 + count on the large-M path; 0 for an invalid or empty shape.  A single
+ * mmf_bitlinear_fwd is count = 1. */
+int mmf_fwd_launches(int64_t M, int64_t K, int64_t N, int count);
+
 /* Bytes of the packed ternary matrix for an N x K weight: N * K / 4. */
 size_t mmf_packed_bytes(int64_t N, int64_t K);
 
 /* Bytes of device workspace mmf_bitlinear_fwd and mmf_ternary_acc need for
- * this shape; 0 when the shape takes the fused decode path (small M), which
- * needs none.  Depends only on (M, K, N). */
+ * this shape; 0 when the shape takes the fused one-token decode path, which
+ * needs none.  For 2 .. 32 tokens it holds the codes in the decode
+ * tensor-core kernel's operand layout (16 or 32 token rows per 128-wide K
+ * chunk) and the per-token absmax and code sums; for more tokens the codes in
+ * row-major order and the same sums.  Depends only on (M, K, N). */
 size_t mmf_workspace_bytes(int64_t M, int64_t K, int64_t N);
 
 /*
@@ -202,7 +212,7 @@ int mmf_mlgru_scan(const uint16_t* f_pre, const uint16_t* c_pre,
  * loaded.  An empty contraction gives zeros (M == 0: dW = 0, dgamma = 0;
  * N == 0: dx = 0).  workspace: at least mmf_bwd_workspace_bytes(M, K, N)
  * bytes, no initialisation needed.  Sizes as the forward, with N a multiple
- * of 8 (dy rows are read by TMA) and M <= 4194240; buffers of an empty extent
+ * of 8 (dy rows are read by TMA), and M <= 4194240 when K > 8192; buffers of an empty extent
  * (x, dx and workspace when M == 0; dW when N == 0; dy and packed when either
  * is 0) may be NULL.
  */

@@ -264,9 +264,10 @@ def test_single_token_matches_large_m_path(oracle, case):
 @pytest.mark.parametrize("M", [2, 3, 5, 8, 13, 16, 17, 24, 32])
 @pytest.mark.parametrize("K", [2560, 6912])
 def test_decode_codes_match_large_m_path(oracle, M, K):
-    """The decode tensor-core path (2 .. 32 tokens) keeps its codes in the MMA's
-    operand layout, with zero rows up to 16 or 32 tokens, and never hands them
-    out.  M tokens on it against the same tokens as the first rows of a
+    """The decode paths never hand their codes out: the CUDA-core kernel (up to
+    8 tokens) forms them in shared memory, the tensor-core one (9 .. 32 tokens)
+    keeps them in the MMA's operand layout with zero rows up to 16 or 32
+    tokens.  M tokens on it against the same tokens as the first rows of a
     64-token batch (codes in row-major order, which the quantiser test compares
     with the oracle, then the large-M tensor-core kernel): bit-equal y means
     equal codes, sums and absmax (a code off by one changes acc for every
@@ -278,8 +279,8 @@ def test_decode_codes_match_large_m_path(oracle, M, K):
     x[0, :] = x[0, :] * 0.0 + 1.5          # a constant token (every |r| ties)
     packed, scale = _pack(W)
     xd, gd = x.to(DEV), g.to(DEV)
-    nt = 16 if M <= 16 else 32               # two different paths: operand layout vs row-major codes
-    assert mmf.workspace_bytes(M, K, N) < nt * K + 1024 < mmf.workspace_bytes(64, K, N)
+    nt = 16 if M <= 16 else 32               # two different paths (codes in shared memory, or in the
+    assert mmf.workspace_bytes(M, K, N) < nt * K + 1024 < mmf.workspace_bytes(64, K, N)   # operand layout)
     y_small = mmf.bitlinear_fwd(xd[:M].contiguous(), gd, packed, scale, N, EPS)
     y_big = mmf.bitlinear_fwd(xd, gd, packed, scale, N, EPS)
     torch.cuda.synchronize()
