@@ -13,7 +13,7 @@
 // Persistent: one CTA per SM walks the tiles (token tile major, weight tile
 // minor, so CTAs working at the same time share activation tiles in L2), with
 // two TMEM accumulators so a tile's epilogue overlaps the next tile's MMAs.
-// Warp roles (768 threads):
+// Warp roles (640 threads):
 //   warp 0      TMA producer: q tile (BT x 128 B, 128-byte swizzle) and the
 //               packed weight tile (128 x 32 B) per stage
 //   warp 1      TMEM allocation; lane 0 issues tcgen05.mma (4 x K=32 per
@@ -22,9 +22,7 @@
 //               the 32 TMEM lanes of sub-partition warp % 4) taking every
 //               third 32-token chunk: tcgen05.ld, subtract sum q, rescale,
 //               transpose through shared memory, 16-byte stores of y
-//   warps 16-23 unpack, two groups of four taking alternate stages (so a
-//               stage's unpack latency overlaps the next one's): thread u of
-//               a group expands row u's 128 codes to int8 in the
+//   warps 16-19 unpack: thread u expands row u's 128 codes to int8 in the
 //               128-byte-swizzled K-major layout the MMA reads
 // Every wait is bounded; on timeout the CTA records the error, drains its
 // copies and MMAs, frees TMEM and exits.
@@ -37,8 +35,7 @@ constexpr int kTcRows = 128;      // weight rows per tile (MMA M)
 constexpr int kTcK = 128;         // K (bytes of int8) per stage
 constexpr int kTcStages = 4;
 constexpr int kTcEpiWarps = 12;                        // three per TMEM sub-partition
-constexpr int kTcUnpackGroups = 2;                     // 4-warp unpack groups taking alternate stages
-constexpr int kTcThreads = (4 + kTcEpiWarps + 4 * kTcUnpackGroups) * 32;  // TMA/MMA/idle, epilogue, unpack
+constexpr int kTcThreads = (8 + kTcEpiWarps) * 32;     // warps 0-3 TMA/MMA/idle, epilogue, 4 unpack
 constexpr int kTcPackedBytes = kTcRows * (kTcK / 4);  // 4 KB of 2-bit codes per stage
 constexpr int kTcEpiBarrier = 2;                       // named barrier of the epilogue warps
 
@@ -182,15 +179,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp >= 4 + kTcEpiWarps) {
         // ------------------------------------------------------------ unpack
-        const int ut = threadIdx.x - (4 + kTcEpiWarps) * 32;
-        const int u = ut & 127;   // weight row within the tile
-        const int ug = ut >> 7;   // this group unpacks stage uses ug, ug + groups, ...
-        static_assert(kTcStages % kTcUnpackGroups == 0, "a stage slot always goes to the same group");
+        const int u = threadIdx.x - (4 + kTcEpiWarps) * 32;  // weight row within the tile
         int g = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += G) {
             for (int ks = 0; ks < nk; ++ks, ++g) {
-                if (g % kTcUnpackGroups != ug) continue;
                 const int s = g % kTcStages;
                 if (!mbar_wait(&full_bar[s], (g / kTcStages) & 1, &abort_flag)) {
                     ok = false;

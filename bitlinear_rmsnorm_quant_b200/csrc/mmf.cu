@@ -265,8 +265,11 @@ mmf_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ba
 template <int BT>
 mmf_status launch_tc_bt(bool fused, const CUtensorMap& mq, const CUtensorMap& mw, TcParams p, cudaStream_t s,
                         bool pdl, int num_sms) {
+    const int64_t tiles = ((static_cast<int64_t>(p.N) + kTcRows - 1) / kTcRows) *
+                          ((static_cast<int64_t>(p.M) + BT - 1) / BT);
+    if (tiles > kMaxDim) return MMF_ERR_UNSUPPORTED_SHAPE;
     p.n_tiles = (p.N + kTcRows - 1) / kTcRows;
-    p.num_tiles = p.n_tiles * ((p.M + BT - 1) / BT);
+    p.num_tiles = static_cast<int>(tiles);
     const dim3 grid(static_cast<unsigned>(p.num_tiles < num_sms ? p.num_tiles : num_sms));  // persistent
     if (fused) return launch(gemm_tc_kernel<BT, true>, grid, dim3(kTcThreads), TcLayout<BT>::smem_bytes, s, pdl, mq, mw, p);
     return launch(gemm_tc_kernel<BT, false>, grid, dim3(kTcThreads), TcLayout<BT>::smem_bytes, s, pdl, mq, mw, p);
