@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) mlgru_scan_kernel(const ui
     // pass 1: the chunk's map h -> A h + B
     float a0 = 1.0f, a1 = 1.0f, b0 = 0.0f, b1 = 0.0f;
     if (valid) {
-#pragma unroll 4
+#pragma unroll 8
         for (int t = t0; t < t1; ++t) {
             float fp0, fp1, cp0, cp1;
             bf16x2_to_f(__ldg(reinterpret_cast<const uint32_t*>(f_pre + idx(t))), fp0, fp1);
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) mlgru_scan_kernel(const ui
 
     // pass 2: the recurrence over the chunk, writing o
     if (valid) {
-#pragma unroll 4
+#pragma unroll 8
         for (int t = t0; t < t1; ++t) {
             float fp0, fp1, cp0, cp1, gp0, gp1;
             bf16x2_to_f(__ldg(reinterpret_cast<const uint32_t*>(f_pre + idx(t))), fp0, fp1);

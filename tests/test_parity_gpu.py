@@ -118,12 +118,13 @@ def test_quantize_special_rows(oracle):
 # -- ternary contraction: int32 bit-exact on the kernel's own q and packed W --------------
 
 ACC_SHAPES = [
-    # (M, K, N) CUDA-core decode kernel (one token)
-    (1, 128, 1), (1, 256, 256), (1, 6912, 20000),   # weight ring refilled many times per CTA
-    # decode tensor-core kernel (2 .. 32 tokens): slabs of 8 .. 128 rows, ragged slabs, the code ring
+    # (M, K, N) CUDA-core decode kernel (1 .. 8 tokens): weight ring refilled many times per CTA
+    (1, 128, 1), (1, 256, 256), (1, 6912, 20000),
+    (2, 1024, 1000), (3, 2560, 333), (8, 6912, 2560), (5, 2816, 1024), (4, 4096, 9000), (2, 128, 8),
+    # decode tensor-core kernel (9 .. 32 tokens): slabs of 8 .. 128 rows, ragged slabs, the code ring
     # refilled (K = 6912: 54 chunks), 16 and 32 operand rows
-    (2, 1024, 1000), (3, 2560, 333), (8, 6912, 2560), (5, 2816, 1024), (4, 4096, 9000), (9, 256, 300),
-    (16, 256, 256), (17, 384, 129), (32, 2560, 640), (32, 6912, 700), (24, 2560, 13824), (2, 128, 8),
+    (9, 256, 300),
+    (16, 256, 256), (17, 384, 129), (32, 2560, 640), (32, 6912, 700), (24, 2560, 13824),
     (31, 8192, 40000),
     # large-M tcgen05 path: several 128-row tiles, token tiles, K stages, ragged tails
     (33, 2048, 500), (100, 1024, 257), (256, 512, 384), (300, 384, 300), (513, 2048, 200),
