@@ -83,44 +83,48 @@ __global__ void __launch_bounds__(kBwdThreads) dgamma_partial_kernel(const uint1
     part[static_cast<int64_t>(blockIdx.y) * K + k] = s;
 }
 
-__global__ void __launch_bounds__(kBwdThreads) dgamma_final_kernel(const double* __restrict__ part, int chunks, int K,
+// Final dgamma stage: a CTA takes 32 columns; its 32 warps sum the partials
+// of chunks w, w + 32, w + 64, ... in order (one column per lane, 256-byte
+// rows per warp), then warp 0 adds the 32 group sums in warp order.
+constexpr int kDgCols = 32;
+constexpr int kDgThreads = 1024;
+constexpr int kDgGroups = kDgThreads / kDgCols;
+
+__global__ void __launch_bounds__(kDgThreads) dgamma_final_kernel(const double* __restrict__ part, int chunks, int K,
                                                                    const float* __restrict__ beta,
                                                                    float* __restrict__ dgamma) {
-    const int k = blockIdx.x * kBwdThreads + threadIdx.x;
-    if (k >= K) return;
+    __shared__ double red[kDgGroups][kDgCols];
+    const int col = threadIdx.x & (kDgCols - 1), grp = threadIdx.x / kDgCols;
+    const int k = blockIdx.x * kDgCols + col;
     double s = 0.0;
-    for (int c = 0; c < chunks; ++c) s += part[static_cast<int64_t>(c) * K + k];
-    dgamma[k] = static_cast<float>(s * static_cast<double>(__ldg(beta)));
+    if (k < K) {
+#pragma unroll 8
+        for (int c = grp; c < chunks; c += kDgGroups) s += __ldg(part + static_cast<int64_t>(c) * K + k);
+    }
+    red[grp][col] = s;
+    __syncthreads();
+    if (grp == 0 && k < K) {
+        double t = 0.0;
+#pragma unroll
+        for (int g = 0; g < kDgGroups; ++g) t += red[g][col];
+        dgamma[k] = static_cast<float>(t * static_cast<double>(__ldg(beta)));
+    }
 }
 
 // RMSNorm backward and the dgamma partial sums in one pass over HBM (K <=
-// 8192): a CTA takes kBwdFusedRows consecutive token rows; thread t owns the
-// 8-column chunks c = t + 256 i (i < CPT) and keeps its columns' dgamma
-// partial sums (fp64) in registers over the CTA's rows.  Per row it reads x
-// and dr (16- and 32-byte loads, kept in L1), forms the row's fp64 sums of
-// x^2 and gamma beta dr x (a warp tree, then the warps in index order), then
-// reads the same lines again from L1 to write dx and add dr x inv to its
-// partials, rows in order.  The CTA's partials go to part[blockIdx.x][k];
+// 8192): a CTA takes kBwdFusedRows consecutive token rows, RPB rows per
+// barrier; thread t owns the 8-column chunks c = t + 256 i (i < CPT), holds
+// their x and dr in registers for the row, and keeps its columns' dgamma
+// partial sums over the CTA's rows.  Per row the sums of x^2 and gamma dr x
+// are fp32 over a thread's columns (x^2 of a bf16 value is exact in fp32),
+// fp64 across the threads (a warp tree, then the warps in index order), and
+// inv, c2 fp64; dx and the partials are formed in fp32 (dx is rounded to bf16
+// once at the end).  The CTA's partials go to part[blockIdx.x][k] (fp64);
 // dgamma_final_kernel sums them over the CTAs in order.
 constexpr int kBwdFusedRows = 16;
 constexpr int kBwdFusedMaxK = kBwdThreads * 8 * 4;
 
-__device__ __forceinline__ void load_x8_dr8(const uint16_t* x, const float* dr, int64_t off, float (&xv)[8],
-                                            float (&dv)[8]) {
-    const uint4 xw = __ldg(reinterpret_cast<const uint4*>(x + off));
-    const float4 da = __ldg(reinterpret_cast<const float4*>(dr + off));
-    const float4 db = __ldg(reinterpret_cast<const float4*>(dr + off) + 1);
-    const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        xv[2 * e] = __uint_as_float(w[e] << 16);
-        xv[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-    }
-    dv[0] = da.x; dv[1] = da.y; dv[2] = da.z; dv[3] = da.w;
-    dv[4] = db.x; dv[5] = db.y; dv[6] = db.z; dv[7] = db.w;
-}
-
-template <int CPT>
+template <int CPT, int RPB>
 __global__ void __launch_bounds__(kBwdThreads) rmsnorm_bwd_fused_kernel(const uint16_t* __restrict__ x,
                                                                         const float* __restrict__ gamma,
                                                                         const float* __restrict__ dr,
@@ -128,77 +132,101 @@ __global__ void __launch_bounds__(kBwdThreads) rmsnorm_bwd_fused_kernel(const ui
                                                                         int K, int64_t M,
                                                                         uint16_t* __restrict__ dx,
                                                                         double* __restrict__ part) {
-    __shared__ double red_s[2][kBwdThreads / 32], red_d[2][kBwdThreads / 32];
+    __shared__ double red[2][RPB][2][kBwdThreads / 32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int C = K >> 3;
     const double bt = static_cast<double>(__ldg(beta));
     const float4* g4 = reinterpret_cast<const float4*>(gamma);
-    double acc[CPT][8];
+    float acc[CPT][8];
 #pragma unroll
     for (int i = 0; i < CPT; ++i)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[i][e] = 0.0;
+        for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
     const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBwdFusedRows;
     const int64_t m1 = m0 + kBwdFusedRows < M ? m0 + kBwdFusedRows : M;
-    for (int64_t m = m0; m < m1; ++m) {
-        const int buf = static_cast<int>(m - m0) & 1;
-        const int64_t row = m * static_cast<int64_t>(K);
-        double s2 = 0.0, dot = 0.0;
+    for (int64_t m = m0; m < m1; m += RPB) {
+        const int buf = static_cast<int>((m - m0) / RPB) & 1;
+        uint4 xw[RPB][CPT];
+        float4 da[RPB][CPT], db[RPB][CPT];
 #pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-            const int c = threadIdx.x + kBwdThreads * i;
-            if (c < C) {
-                float xv[8], dv[8];
-                load_x8_dr8(x, dr, row + 8 * c, xv, dv);
-                const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
-                const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+        for (int r = 0; r < RPB; ++r)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const double xd = xv[e];
-                    s2 += xd * xd;
-                    dot += static_cast<double>(g[e]) * (bt * static_cast<double>(dv[e])) * xd;
+            for (int i = 0; i < CPT; ++i) {
+                const int c = threadIdx.x + kBwdThreads * i;
+                if (c < C && m + r < m1) {
+                    const int64_t off = (m + r) * static_cast<int64_t>(K) + 8 * c;
+                    xw[r][i] = __ldg(reinterpret_cast<const uint4*>(x + off));
+                    da[r][i] = __ldg(reinterpret_cast<const float4*>(dr + off));
+                    db[r][i] = __ldg(reinterpret_cast<const float4*>(dr + off) + 1);
+                } else {
+                    xw[r][i] = make_uint4(0u, 0u, 0u, 0u);
+                    da[r][i] = db[r][i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 }
             }
-        }
-        s2 = warp_sum_f64(s2);
-        dot = warp_sum_f64(dot);
-        if (lane == 0) {
-            red_s[buf][warp] = s2;
-            red_d[buf][warp] = dot;
-        }
-        __syncthreads();  // (the other buffer was last read before the previous row's barrier)
-        s2 = 0.0;
-        dot = 0.0;
 #pragma unroll
-        for (int w = 0; w < kBwdThreads / 32; ++w) {
-            s2 += red_s[buf][w];
-            dot += red_d[buf][w];
-        }
-        const double inv = 1.0 / sqrt(s2 / static_cast<double>(K) + static_cast<double>(eps));
-        const double c2 = inv * inv * inv * dot / static_cast<double>(K);
+        for (int r = 0; r < RPB; ++r) {
+            float s2 = 0.0f, dot = 0.0f;
 #pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-            const int c = threadIdx.x + kBwdThreads * i;
-            if (c < C) {
-                float xv[8], dv[8];
-                load_x8_dr8(x, dr, row + 8 * c, xv, dv);
-                const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
-                const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-                uint32_t o[4];
+            for (int i = 0; i < CPT; ++i) {
+                const int c = threadIdx.x + kBwdThreads * i;
+                if (c < C) {
+                    float xv[8];
+                    unpack_bf16x8(xw[r][i], xv);
+                    const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
+                    const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                    const float d[8] = {da[r][i].x, da[r][i].y, da[r][i].z, da[r][i].w,
+                                        db[r][i].x, db[r][i].y, db[r][i].z, db[r][i].w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    uint32_t h[2];
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int k = 2 * e + j;
-                        const double xd = xv[k], drd = static_cast<double>(dv[k]);
-                        const double gr = inv * static_cast<double>(g[k]) * (bt * drd) - xd * c2;
-                        h[j] = __bfloat16_as_ushort(__double2bfloat16(gr));
-                        acc[i][k] += drd * xd * inv;
+                    for (int e = 0; e < 8; ++e) {
+                        s2 = fmaf(xv[e], xv[e], s2);
+                        dot = fmaf(g[e] * d[e], xv[e], dot);
                     }
-                    o[e] = h[0] | (h[1] << 16);
                 }
-                *reinterpret_cast<uint4*>(dx + row + 8 * c) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            const double s2w = warp_sum_f64(static_cast<double>(s2));
+            const double dotw = warp_sum_f64(static_cast<double>(dot));
+            if (lane == 0) {
+                red[buf][r][0][warp] = s2w;
+                red[buf][r][1][warp] = dotw;
+            }
+        }
+        __syncthreads();  // (the other buffer was last read before the previous barrier)
+#pragma unroll
+        for (int r = 0; r < RPB; ++r) {
+            double s2 = 0.0, dot = 0.0;
+#pragma unroll
+            for (int w = 0; w < kBwdThreads / 32; ++w) {
+                s2 += red[buf][r][0][w];
+                dot += red[buf][r][1][w];
+            }
+            const double inv = 1.0 / sqrt(s2 / static_cast<double>(K) + static_cast<double>(eps));
+            const float c2 = static_cast<float>(inv * inv * inv * (bt * dot) / static_cast<double>(K));
+            const float ib = static_cast<float>(inv * bt), invf = static_cast<float>(inv);
+            if (m + r < m1) {
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) {
+                    const int c = threadIdx.x + kBwdThreads * i;
+                    if (c < C) {
+                        float xv[8];
+                        unpack_bf16x8(xw[r][i], xv);
+                        const float4 ga = __ldg(g4 + 2 * c), gb = __ldg(g4 + 2 * c + 1);
+                        const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                        const float d[8] = {da[r][i].x, da[r][i].y, da[r][i].z, da[r][i].w,
+                                            db[r][i].x, db[r][i].y, db[r][i].z, db[r][i].w};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float v0 = fmaf(ib * g[2 * e], d[2 * e], -xv[2 * e] * c2);
+                            const float v1 = fmaf(ib * g[2 * e + 1], d[2 * e + 1], -xv[2 * e + 1] * c2);
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+                            o[e] = *reinterpret_cast<const uint32_t*>(&h);
+                            acc[i][2 * e] = fmaf(d[2 * e] * xv[2 * e], invf, acc[i][2 * e]);
+                            acc[i][2 * e + 1] = fmaf(d[2 * e + 1] * xv[2 * e + 1], invf, acc[i][2 * e + 1]);
+                        }
+                        *reinterpret_cast<uint4*>(dx + (m + r) * static_cast<int64_t>(K) + 8 * c) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
             }
         }
     }
@@ -208,7 +236,7 @@ __global__ void __launch_bounds__(kBwdThreads) rmsnorm_bwd_fused_kernel(const ui
         if (c < C) {
             double* pr = part + static_cast<int64_t>(blockIdx.x) * K + 8 * c;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) pr[e] = acc[i][e];
+            for (int e = 0; e < 8; ++e) pr[e] = static_cast<double>(acc[i][e]);
         }
     }
 }

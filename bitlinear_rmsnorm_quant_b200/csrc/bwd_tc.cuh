@@ -266,13 +266,27 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         const int part = t & 3;              // quarter of the 128 k
         int g = 0;
         bool ok = true;
+        // dW: token j's absmax of stage ks depends on ks alone (every tile runs the same
+        // contraction), so each thread loads it two stages ahead and the load's latency
+        // stays off the conversion
+        const auto absmax_at = [&](int ks) -> float {
+            const int m = ks * kBwKs + j;
+            return m < p.contr ? __ldg(p.absmax + m) : 0.0f;
+        };
+        float am_cur = 0.0f, am_next = 0.0f;
+        if constexpr (MODE == 1) {
+            am_cur = absmax_at(0);
+            am_next = absmax_at(nk > 1 ? 1 : 0);
+        }
         for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += G) {
             for (int ks = 0; ks < nk; ++ks, ++g) {
                 const int s = g % kBwStages;
                 float sc = 0.0f;
                 if constexpr (MODE == 1) {
-                    const int m = ks * kBwKs + j;
-                    if (m < p.contr) sc = __fdiv_rn(__ldg(p.absmax + m), 127.0f);
+                    const float am_far = absmax_at((ks + 2) % nk);
+                    sc = __fdiv_rn(am_cur, 127.0f);
+                    am_cur = am_next;
+                    am_next = am_far;
                 }
                 if (!mbar_wait(&full_bar[s], (g / kBwStages) & 1, &abort_flag)) {
                     ok = false;

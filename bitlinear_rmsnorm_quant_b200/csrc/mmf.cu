@@ -112,6 +112,7 @@ mmf_status device_state(DeviceState** out) {
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8, true>, 2 * kMaxK);
         if (e == cudaSuccess) e = set_smem(gemm_bwd_kernel<0>, BwLayout<0>::smem_bytes);
         if (e == cudaSuccess) e = set_smem(gemm_bwd_kernel<1>, BwLayout<1>::smem_bytes);
+        if (e == cudaSuccess) e = set_smem(mlgru_scan_tma_kernel, kStSmemBytes);
         if (e != cudaSuccess) return MMF_ERR_CUDA;
         if (!g_encode_tiled) {
             void* fn = nullptr;
@@ -703,10 +704,10 @@ int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma,
         // dx and the dgamma partials in one pass over x and dr
         const int cpt = static_cast<int>((K / 8 + kBwdThreads - 1) / kBwdThreads);  // 1, 2, 3 or 4
         void (*kern)(const uint16_t*, const float*, const float*, const float*, float, int, int64_t, uint16_t*,
-                     double*) = cpt == 1   ? rmsnorm_bwd_fused_kernel<1>
-                                : cpt == 2 ? rmsnorm_bwd_fused_kernel<2>
-                                : cpt == 3 ? rmsnorm_bwd_fused_kernel<3>
-                                           : rmsnorm_bwd_fused_kernel<4>;
+                     double*) = cpt == 1   ? rmsnorm_bwd_fused_kernel<1, 2>
+                                : cpt == 2 ? rmsnorm_bwd_fused_kernel<2, 2>
+                                : cpt == 3 ? rmsnorm_bwd_fused_kernel<3, 1>
+                                           : rmsnorm_bwd_fused_kernel<4, 1>;
         if ((st = launch(kern, dim3(static_cast<unsigned>(chunks)), dim3(kBwdThreads), 0, s, false, x, gamma,
                          static_cast<const float*>(dr), scale, eps, static_cast<int>(K), M, dx, part)) != MMF_OK)
             return st;
@@ -719,7 +720,8 @@ int mmf_bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const float* gamma,
                          static_cast<int>(K), part)) != MMF_OK)
             return st;
     }
-    return launch(dgamma_final_kernel, blocks(K), dim3(kBwdThreads), 0, s, false, static_cast<const double*>(part), chunks,
+    return launch(dgamma_final_kernel, dim3(static_cast<unsigned>((K + kDgCols - 1) / kDgCols)), dim3(kDgThreads), 0, s,
+                  false, static_cast<const double*>(part), chunks,
                   static_cast<int>(K), scale, dgamma);
 }
 
@@ -738,6 +740,20 @@ int mmf_mlgru_scan(const uint16_t* f_pre, const uint16_t* c_pre, const uint16_t*
     mmf_status st = device_state(&dev);
     if (st != MMF_OK) return st;
     const dim3 grid(static_cast<unsigned>((D + 63) / 64), static_cast<unsigned>(B));
+    const int64_t rows = B * T;
+    if (T > 0 && D % 8 == 0 && D >= kStCh && rows >= kStRows && rows <= int64_t(INT32_MAX) - kStRows) {
+        // tensor maps over the [B * T][D] pre-activations: 64 channels x 128 tokens per copy
+        CUtensorMap mf, mc, mg;
+        if ((st = encode_2d(&mf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f_pre, D, rows, 2 * D, kStCh, kStRows,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)) != MMF_OK ||
+            (st = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c_pre, D, rows, 2 * D, kStCh, kStRows,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)) != MMF_OK ||
+            (st = encode_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g_pre, D, rows, 2 * D, kStCh, kStRows,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)) != MMF_OK)
+            return st;
+        return launch(mlgru_scan_tma_kernel, grid, dim3(kStThreads), kStSmemBytes, static_cast<cudaStream_t>(stream),
+                      false, mf, mc, mg, h0, static_cast<int>(T), static_cast<int>(D), o, h_last);
+    }
     return launch(mlgru_scan_kernel, grid, dim3(kScanWarps * 32), 0, static_cast<cudaStream_t>(stream), false, f_pre,
                   c_pre, g_pre, h0, static_cast<int>(T), static_cast<int>(D), o, h_last);
 }

@@ -46,16 +46,6 @@ struct AddOp {
     __device__ __forceinline__ T operator()(T a, T b) const { return a + b; }
 };
 
-// 8 bf16 in a uint4 -> 8 floats
-__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float (&f)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
-
 // Byte offset of codes k = 8 c8 .. 8 c8 + 7 of token m in the decode
 // tensor-core kernel's B layout for NT token rows: per 128-wide K chunk, NT
 // rows of 128 bytes in 8-row 1024-byte atoms, 16-byte units swizzled by the

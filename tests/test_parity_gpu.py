@@ -378,8 +378,12 @@ def test_glu_paths_agree_and_match_plain_call():
 
 # -- MLGRU token mixer recurrence -------------------------------------------------------------
 
-@pytest.mark.parametrize("B,T,D", [(1, 1, 2560), (2, 37, 128), (3, 100, 66), (4, 2048, 2048), (2, 5, 64),
-                                   (1, 0, 64)])
+@pytest.mark.parametrize("B,T,D", [
+    # per-warp chunk kernel: few rows, D not a multiple of 8, no tokens
+    (1, 1, 2560), (2, 37, 128), (3, 100, 66), (2, 5, 64), (1, 0, 64),
+    # tensor-copy kernel: 128-token stages, ragged last stage (the next sequence's rows
+    # read and ignored), channels past D in the last CTA, sequences shorter than a stage
+    (4, 2048, 2048), (2, 300, 200), (1, 1000, 4104), (5, 70, 512), (3, 128, 64)])
 @pytest.mark.parametrize("with_h0", [False, True])
 def test_mlgru_scan_parity(oracle, B, T, D, with_h0):
     rng = np.random.default_rng(B * 1000 + T + D)
