@@ -333,10 +333,19 @@ mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_
     // persistent: rows in registers, WPR warps per row (K <= 2048 WPR), as many
     // CTAs as fit on the SMs at once, never more than the rows need
     const int wpr = static_cast<int>((K + 2047) / 2048);
-    void (*kern)(const uint16_t*, const float*, float, int, int64_t, int8_t*, float*, int*) =
-        wpr == 1 ? rmsnorm_quant_reg_kernel<1>
-                 : (wpr == 2 ? rmsnorm_quant_reg_kernel<2>
-                             : (wpr == 3 ? rmsnorm_quant_reg_kernel<3> : rmsnorm_quant_reg_kernel<4>));
+    // 16-byte chunks a lane holds: as few as the width needs (fewer registers
+    // for the row and its successor in flight)
+    const int ch = static_cast<int>((K / 8 + 32 * wpr - 1) / (32 * wpr));
+    using QuantRegFn = void (*)(const uint16_t*, const float*, float, int, int64_t, int8_t*, float*, int*);
+    QuantRegFn kern;
+    switch (wpr) {
+        case 1: kern = ch <= 4 ? rmsnorm_quant_reg_kernel<1, 4> : ch <= 6 ? rmsnorm_quant_reg_kernel<1, 6>
+                                                                          : rmsnorm_quant_reg_kernel<1, 8>; break;
+        case 2: kern = ch <= 5 ? rmsnorm_quant_reg_kernel<2, 5> : ch <= 6 ? rmsnorm_quant_reg_kernel<2, 6>
+                                                                          : rmsnorm_quant_reg_kernel<2, 8>; break;
+        case 3: kern = rmsnorm_quant_reg_kernel<3, 8>; break;
+        default: kern = ch <= 7 ? rmsnorm_quant_reg_kernel<4, 7> : rmsnorm_quant_reg_kernel<4, 8>; break;
+    }
     const int threads = quant_reg_warps(wpr) * 32;
     const int rpc = quant_reg_warps(wpr) / wpr;
     const size_t smem = static_cast<size_t>(K) * 4;

@@ -225,18 +225,18 @@ __global__ void __launch_bounds__(kQuantCtaWarps * 32) rmsnorm_quant_kernel(cons
 // the definition never changes a code.  Four bytes are packed with byte
 // permutes and summed with one DP4A.  The reductions are a fixed warp tree,
 // then the group's warps in index order.
-constexpr int kQuantRegChunks = 8;       // 16-byte chunks of x per lane per row
+constexpr int kQuantRegChunks = 8;       // most 16-byte chunks of x a lane holds per row (CHT)
 constexpr int kMaxQuantRegK = 8192;      // WPR <= 4
 
 __host__ __device__ constexpr int quant_reg_warps(int WPR) { return WPR == 3 ? 6 : 8; }
 
-template <int WPR>
+template <int WPR, int CHT = 8>
 __global__ void __launch_bounds__(quant_reg_warps(WPR) * 32, 2) rmsnorm_quant_reg_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ gamma, float eps, int K, int64_t M,
     int8_t* __restrict__ q, float* __restrict__ absmax, int* __restrict__ qsum) {
     constexpr int NW = quant_reg_warps(WPR);
     constexpr int RPC = NW / WPR;  // row groups per CTA
-    constexpr int CH = kQuantRegChunks;
+    constexpr int CH = CHT;
     extern __shared__ __align__(16) float4 gamma_s[];  // K / 4
     __shared__ double red_d[NW];
     __shared__ float red_f[NW];
