@@ -778,6 +778,14 @@ def run_workload(name, args, dist, steps, warmup, peaks, peak_src, copy_gbs=None
                         "of this kernel are in the profiles, not measured in this run"}
     if split:
         roof["split"] = split
+    if roof["bound"] == "tensor":
+        # context: the datasheet's dense int8 figure over the whole step, and a
+        # library int8 GEMM (8192^3) on this GPU, timed after this workload
+        roof["step_frac_of_datasheet_4500"] = round(step_achieved / 4500.0, 4)
+        lib_tops = library_int8_tops()
+        roof["library_int8_gemm_tops"] = lib_tops
+        if isinstance(lib_tops, float):
+            roof["frac_of_library_int8_gemm"] = round(achieved / lib_tops, 4)
     res = {
         "metric": METRIC, "value": round(value, 2),
         "unit": "tokens/s (one token through one BitLinear layer set)",

@@ -406,6 +406,34 @@ def test_mlgru_scan_parity(oracle, B, T, D, with_h0):
         assert (ov == rv).mean() > 0.99
 
 
+@pytest.mark.parametrize("B,T,D", [(2, 300, 128), (1, 129, 66)])
+def test_mlgru_scan_saturated_gates(oracle, B, T, D):
+    """Pre-activations of +-60 mixed into normal ones: gates at 0 and 1 within
+    fp32, the SiLU input large on both sides; the tensor-copy kernel (D = 128)
+    and the per-warp-chunk one (D = 66).  The kernels clamp pre-activations at
+    -28 before the exponential, so a gate of sigma(-60) = 9e-27 comes out as
+    sigma(-28) = 7e-13: o then differs from the oracle's by far less than the
+    absolute bound, though not bit for bit, so bit equality is counted over
+    the outputs above 1e-6."""
+    rng = np.random.default_rng(B * 7 + T + D)
+    v = lambda: rng.standard_normal((B, T, D)).astype(np.float32) * 2.0
+    fp, cp, gp = v(), v(), v()
+    for a in (fp, cp, gp):
+        a[rng.random(a.shape) < 0.1] = 60.0
+        a[rng.random(a.shape) < 0.1] = -60.0
+    bf = lambda a: torch.from_numpy(a).to(torch.bfloat16)
+    fb, cb, gb = bf(fp), bf(cp), bf(gp)
+    o, hl = mmf.mlgru_scan(fb.to(DEV), cb.to(DEV), gb.to(DEV), None)
+    torch.cuda.synchronize()
+    o_ref, hl_ref = oracle.mlgru_scan(bits_np(fb), bits_np(cb), bits_np(gb), None)
+    ov, rv = bf16_to_f64(bits_np(o.cpu())), bf16_to_f64(o_ref)
+    assert np.isfinite(ov).all()
+    assert (np.abs(hl.cpu().numpy() - hl_ref) <= 1e-4 * (1.0 + np.abs(hl_ref))).all()
+    assert (np.abs(ov - rv) <= np.abs(rv) * 2.0 ** -7 + 1e-6).all()
+    big = np.abs(rv) >= 1e-6
+    assert big.mean() > 0.5 and (ov[big] == rv[big]).mean() > 0.99
+
+
 def test_mlgru_scan_continues_across_calls():
     """Two calls over the halves of the tokens, the state carried, give the
     single call's output to fp32 rounding of the state."""
