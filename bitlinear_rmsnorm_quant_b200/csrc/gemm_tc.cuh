@@ -13,6 +13,9 @@
 // Persistent: one CTA per SM walks the tiles (token tile major, weight tile
 // minor, so CTAs working at the same time share activation tiles in L2), with
 // two TMEM accumulators so a tile's epilogue overlaps the next tile's MMAs.
+// When the tiles end in a partial wave of R tiles with 2R <= the grid, those
+// tiles become 2R items of BT / 2 tokens each (an N = BT / 2 MMA on the first
+// half of the loaded token tile), so the last wave takes half a tile's time.
 // Warp roles (640 threads):
 //   warp 0      TMA producer: q tile (BT x 128 B, 128-byte swizzle) and the
 //               packed weight tile (128 x 32 B) per stage
@@ -59,6 +62,10 @@ struct TcParams {
     int M, K, N;
     int n_tiles;            // ceil(N / 128)
     int num_tiles;          // n_tiles * ceil(M / BT)
+    // work items: the first full_items are whole tiles; each tile after them
+    // (the last, partial wave) is two items of BT / 2 tokens (BT = 256 only)
+    int full_items;
+    int num_items;
 };
 
 template <int BT, bool FUSED>
@@ -88,6 +95,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nk = p.K / kTcK;
     const int G = gridDim.x;
+    // work item -> weight rows n0.., tokens t0 .. t0 + ntok - 1
+    auto item_at = [&](int it, int& n0, int& t0, int& ntok) {
+        int tile = it, hv = 0;
+        ntok = BT;
+        if (it >= p.full_items) {
+            tile = p.full_items + ((it - p.full_items) >> 1);
+            hv = (it - p.full_items) & 1;
+            ntok = BT / 2;
+        }
+        n0 = (tile % p.n_tiles) * kTcRows;
+        t0 = (tile / p.n_tiles) * BT + hv * (BT / 2);
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kTcStages; ++s) {
@@ -123,9 +142,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             int g = 0;  // stage uses so far
             bool ok = true;
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += G) {
-                const int n0 = (tile % p.n_tiles) * kTcRows;
-                const int t0 = (tile / p.n_tiles) * BT;
+            for (int it = blockIdx.x; it < p.num_items && ok; it += G) {
+                int n0, t0, ntok;
+                item_at(it, n0, t0, ntok);  // a half item loads the whole box from t0 (rows past M read zero)
                 for (int ks = 0; ks < nk; ++ks, ++g) {
                     const int s = g % kTcStages;
                     if (g >= kTcStages && !mbar_wait(&empty_bar[s], ((g / kTcStages) - 1) & 1, &abort_flag)) {
@@ -145,10 +164,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_i8(kTcRows, BT);
+            constexpr uint32_t idesc_full = idesc_i8(kTcRows, BT);
+            constexpr uint32_t idesc_half = BT == 256 ? idesc_i8(kTcRows, BT / 2) : idesc_full;
             bool issued_any = false, ok = true;
             int g = 0, li = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += G, ++li) {
+            for (int it = blockIdx.x; it < p.num_items && ok; it += G, ++li) {
+                const uint32_t idesc = it < p.full_items ? idesc_full : idesc_half;  // N = the item's tokens
                 const int buf = li & 1;
                 if (li >= 2 && !mbar_wait(&tempty_bar[buf], ((li >> 1) - 1) & 1, &abort_flag)) break;
                 tc_fence_after();
@@ -182,7 +203,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int u = threadIdx.x - (4 + kTcEpiWarps) * 32;  // weight row within the tile
         int g = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += G) {
+        for (int it = blockIdx.x; it < p.num_items && ok; it += G) {
             for (int ks = 0; ks < nk; ++ks, ++g) {
                 const int s = g % kTcStages;
                 if (!mbar_wait(&full_bar[s], (g / kTcStages) & 1, &abort_flag)) {
@@ -217,13 +238,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint16_t* stg = epi_tile + (warp - 4) * (16 * 32);  // [16 tokens][32 rows] bf16
         const bool vec_ok = FUSED && (p.N % 8) == 0;
         int li = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += G, ++li) {
+        for (int it = blockIdx.x; it < p.num_items; it += G, ++li) {
             const int buf = li & 1;
-            const int n0 = (tile % p.n_tiles) * kTcRows;
-            const int t0 = (tile / p.n_tiles) * BT;
+            int n0, t0, ntok;
+            item_at(it, n0, t0, ntok);
             // per-token constants of this tile (the previous tile's are no longer read)
             asm volatile("bar.sync %0, %1;" ::"n"(kTcEpiBarrier), "n"(kTcEpiWarps * 32) : "memory");
-            for (int i = et; i < BT; i += kTcEpiWarps * 32) {
+            for (int i = et; i < ntok; i += kTcEpiWarps * 32) {
                 const int t = t0 + i;
                 int qs = 0;
                 float cm = 0.0f;
@@ -239,10 +260,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!named_barrier_and<kTcEpiBarrier, kTcEpiWarps * 32>(got)) break;
             tc_fence_after();
             const int n = n0 + 32 * wq + lane;
-            constexpr int kChunks = BT < 32 ? 1 : BT / 32;
+            const int chunks = BT < 32 ? 1 : ntok / 32;
             constexpr int kCols = BT < 32 ? BT : 32;
 #pragma unroll 1
-            for (int cc = half; cc < kChunks; cc += kTcEpiWarps / 4) {
+            for (int cc = half; cc < chunks; cc += kTcEpiWarps / 4) {
                 uint32_t r[32];
                 const uint32_t taddr = tmem_base + static_cast<uint32_t>(buf * L::acc_cols) +
                                        (static_cast<uint32_t>(32 * wq) << 16) + 32 * cc;

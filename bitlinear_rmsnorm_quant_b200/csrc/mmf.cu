@@ -271,7 +271,18 @@ mmf_status launch_tc_bt(bool fused, const CUtensorMap& mq, const CUtensorMap& mw
     if (tiles > kMaxDim) return MMF_ERR_UNSUPPORTED_SHAPE;
     p.n_tiles = (p.N + kTcRows - 1) / kTcRows;
     p.num_tiles = static_cast<int>(tiles);
-    const dim3 grid(static_cast<unsigned>(p.num_tiles < num_sms ? p.num_tiles : num_sms));  // persistent
+    // the last, partial wave of R tiles as 2R half-token items when they fit
+    // one wave (each CTA then spends half a tile there instead of a tile)
+    p.full_items = p.num_tiles;
+    p.num_items = p.num_tiles;
+    if (BT == 256) {
+        const int rem = p.num_tiles % num_sms;
+        if (rem > 0 && 2 * rem <= num_sms) {
+            p.full_items = p.num_tiles - rem;
+            p.num_items = p.full_items + 2 * rem;
+        }
+    }
+    const dim3 grid(static_cast<unsigned>(p.num_items < num_sms ? p.num_items : num_sms));  // persistent
     if (fused) return launch(gemm_tc_kernel<BT, true>, grid, dim3(kTcThreads), TcLayout<BT>::smem_bytes, s, pdl, mq, mw, p);
     return launch(gemm_tc_kernel<BT, false>, grid, dim3(kTcThreads), TcLayout<BT>::smem_bytes, s, pdl, mq, mw, p);
 }
