@@ -26,7 +26,12 @@
 //               (4 x K = 32 per chunk) and the commits
 //   warps 4-7   epilogue: tcgen05.ld of the 128 x NT accumulator, subtract
 //               sum q, rescale, bf16 y (a warp's 32 lanes = 32 rows)
-//   warps 8-15  unpack: 2-bit codes of the slab -> int8 A tile per chunk
+//   warps 8-15  unpack: 2-bit codes of the slab -> int8 A tiles
+// The unpack warps and the MMA thread hand over units of two chunks (a
+// barrier wait costs about as much as issuing four small MMAs): per unit the
+// unpack warps write two A tiles, make sure the unit's code chunks have
+// landed, and signal the unit full once; the MMA thread waits once, issues 8
+// MMAs and commits the unit's A slot and its two code slots.
 // Every wait is bounded; on timeout the CTA records the error, drains its
 // copies and MMAs, frees TMEM and exits.
 #pragma once
@@ -38,6 +43,8 @@ constexpr int kGtRows = 128;                 // A rows per CTA (MMA M)
 constexpr int kGtThreads = 16 * 32;
 constexpr int kGtUnpackThreads = 256;        // warps 8-15
 constexpr int kGtASlots = 4;                 // unpacked weight chunks in flight
+constexpr int kGtUnit = 2;                   // chunks per unpack/MMA hand-over
+constexpr int kGtUnits = kGtASlots / kGtUnit;
 constexpr int kGtMaxBSlots = 32;
 constexpr int kGtMaxProj = 8;
 constexpr int kGtSmemBudget = 220 * 1024;
@@ -108,8 +115,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     static_assert(NT == 16 || NT == 32, "MMA N is 16 or 32 tokens");
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t w_bar;
-    __shared__ __align__(8) uint64_t a_full[kGtASlots];
-    __shared__ __align__(8) uint64_t a_empty[kGtASlots];
+    __shared__ __align__(8) uint64_t a_full[kGtUnits];
+    __shared__ __align__(8) uint64_t a_empty[kGtUnits];
     __shared__ __align__(8) uint64_t b_full[kGtMaxBSlots];
     __shared__ __align__(8) uint64_t b_empty[kGtMaxBSlots];
     __shared__ __align__(8) uint64_t d_full;
@@ -138,7 +145,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
 
     if (threadIdx.x == 0) {
         mbar_init(&w_bar, 1);
-        for (int s = 0; s < kGtASlots; ++s) {
+        for (int s = 0; s < kGtUnits; ++s) {
             mbar_init(&a_full[s], kGtUnpackThreads);
             mbar_init(&a_empty[s], 1);
         }
@@ -193,20 +200,24 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_i8(kGtRows, NT);
             bool issued = false;
-            for (int c = 0; c < nchunks; ++c) {
-                const int sa = c % kGtASlots, sb = c % S;
-                if (!mbar_wait(&a_full[sa], (c / kGtASlots) & 1, &abort_flag) ||
-                    !mbar_wait(&b_full[sb], (c / S) & 1, &abort_flag))
-                    break;
+            const int nunits = (nchunks + kGtUnit - 1) / kGtUnit;
+            for (int u = 0; u < nunits; ++u) {
+                const int su = u % kGtUnits;
+                // a full unit also means its code chunks have landed (the unpack warps waited)
+                if (!mbar_wait(&a_full[su], (u / kGtUnits) & 1, &abort_flag)) break;
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(a_base + sa * kABytes), b0 = smem_u32(b_base + sb * kBBytes);
+                const int c0 = kGtUnit * u, c1 = min(c0 + kGtUnit, nchunks);
+                for (int c = c0; c < c1; ++c) {
+                    const uint32_t a0 = smem_u32(a_base + (kGtUnit * su + c - c0) * kABytes);
+                    const uint32_t b0 = smem_u32(b_base + (c % S) * kBBytes);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_i8(tmem_base, sw128_kmajor_desc(a0 + 32 * kk), sw128_kmajor_desc(b0 + 32 * kk), idesc,
-                           (c | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_i8(tmem_base, sw128_kmajor_desc(a0 + 32 * kk), sw128_kmajor_desc(b0 + 32 * kk), idesc,
+                               (c | kk) != 0 ? 1u : 0u);
+                }
                 issued = true;
-                mma_commit(&a_empty[sa]);
-                mma_commit(&b_empty[sb]);
+                mma_commit(&a_empty[su]);
+                for (int c = c0; c < c1; ++c) mma_commit(&b_empty[c % S]);
             }
             if (issued) mma_commit(&d_full);
             if (issued && abort_flag) {  // d_full may never be waited on: let the MMAs drain here
@@ -229,10 +240,13 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             }
         }
         const bool got_w = mbar_wait(&w_bar, 0, &abort_flag);
-        for (int c = 0; c < nchunks && got_w; ++c) {
-            const int sa = c % kGtASlots;
-            if (c >= kGtASlots && !mbar_wait(&a_empty[sa], ((c / kGtASlots) - 1) & 1, &abort_flag)) break;
-            if (row < nrows) {
+        const int nunits = (nchunks + kGtUnit - 1) / kGtUnit;
+        for (int u = 0; u < nunits && got_w; ++u) {
+            const int su = u % kGtUnits;
+            if (u >= kGtUnits && !mbar_wait(&a_empty[su], ((u / kGtUnits) - 1) & 1, &abort_flag)) break;
+            const int c0 = kGtUnit * u, c1 = min(c0 + kGtUnit, nchunks);
+            for (int c = c0; c < c1 && row < nrows; ++c) {
+                const int sa = kGtUnit * su + c - c0;
                 // words 4 half .. 4 half + 3 of the chunk: K bytes 16 (4 half + i) .. + 15
                 const uint4 wv = *reinterpret_cast<const uint4*>(w_s + static_cast<size_t>(row) * rowbytes + 32 * c +
                                                                  16 * half);
@@ -247,7 +261,11 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                 }
             }
             fence_proxy_async_smem();
-            mbar_arrive(&a_full[sa]);
+            // the unit's code chunks: landed before the unit is signalled full
+            bool bok = true;
+            if (lane < c1 - c0) bok = mbar_wait(&b_full[(c0 + lane) % S], ((c0 + lane) / S) & 1, &abort_flag);
+            if (!__all_sync(0xffffffffu, bok)) break;
+            mbar_arrive(&a_full[su]);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue
