@@ -391,12 +391,12 @@ def proj_ops(M, K, N):
 def contraction_kernel(mmf, wl) -> str:
     """The kernel that contracts this workload's tokens with the weights, as
     the library dispatches it: the fused decode kernel (normalisation in the
-    same launch, no workspace), the decode tensor-core kernel (9 .. 32 tokens)
+    same launch, no workspace), the decode tensor-core kernel (4 .. 32 tokens)
     or the large-M tensor-core kernel."""
     p = wl.projections[0]
     if mmf.workspace_bytes(wl.M, p.K, p.N) == 0:
         return "gemv_kernel"
-    return "gemv_tc_kernel" if wl.M <= 32 else "gemm_tc_kernel"
+    return "gemv_wide_kernel" if wl.M <= 32 else "gemm_tc_kernel"
 
 
 def hbm_bound(wl) -> bool:
@@ -716,7 +716,7 @@ def run_workload(name, args, dist, steps, warmup, peaks, peak_src, copy_gbs=None
     e2e_value = tokens_per_step / (e2e_ms / 1e3)
     kernel = contraction_kernel(st.mmf, wl)
     # the dominant kernel's own time: the step minus its quantiser launches,
-    # which are timed alone in a graph of their own (none below 9 tokens, where
+    # which are timed alone in a graph of their own (none below 4 tokens, where
     # the decode kernel normalises and quantises in the same launch)
     split = None
     if kernel != "gemv_kernel" and not args.glu:

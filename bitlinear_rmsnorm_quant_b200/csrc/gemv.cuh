@@ -43,7 +43,7 @@ __host__ __device__ constexpr int gemv_compute_warps(int) { return 8; }
 __host__ __device__ constexpr int gemv_threads(int M) { return (gemv_compute_warps(M) + 1) * 32; }
 __host__ __device__ constexpr int gemv_ctas_per_sm(int M) { return M <= 4 ? 2 : 1; }
 constexpr int kGemvMaxStages = 8;
-constexpr int kGemvMaxTokens = 8;
+constexpr int kGemvMaxTokens = 3;  // from 4 tokens the decode tensor-core kernel is faster
 constexpr int kGemvMaxProj = 8;
 constexpr int kGemvStageTarget = 10240;      // bytes of packed weights per stage
 constexpr int kGemvBlockRows = 8;            // rows per warp work item

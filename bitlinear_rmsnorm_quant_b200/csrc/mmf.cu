@@ -12,7 +12,7 @@
 #include "copy.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
-#include "gemv_tc.cuh"
+#include "gemv_wide.cuh"
 #include "pack.cuh"
 #include "quant.cuh"
 #include "scan.cuh"
@@ -30,6 +30,7 @@ constexpr int64_t kMaxK = 65536;  // the quantiser stages one bf16 row (2K bytes
 struct DeviceState {
     bool ready = false;
     int num_sms = 0;
+    int wide_clusters[kGwMaxCluster + 1] = {};  // clusters of k decode tensor-core CTAs resident at once
 };
 
 std::mutex g_mu;
@@ -96,24 +97,40 @@ mmf_status device_state(DeviceState** out) {
         if (e == cudaSuccess) e = set_tc_attrs<64>();
         if (e == cudaSuccess) e = set_tc_attrs<128>();
         if (e == cudaSuccess) e = set_tc_attrs<256>();
-        if (e == cudaSuccess) e = set_smem(gemv_tc_kernel<16, true>, kGtSmemBudget);
-        if (e == cudaSuccess) e = set_smem(gemv_tc_kernel<16, false>, kGtSmemBudget);
-        if (e == cudaSuccess) e = set_smem(gemv_tc_kernel<32, true>, kGtSmemBudget);
-        if (e == cudaSuccess) e = set_smem(gemv_tc_kernel<32, false>, kGtSmemBudget);
+        if (e == cudaSuccess) e = set_smem(gemv_wide_kernel<16, true>, kGwSmemBudget);
+        if (e == cudaSuccess) e = set_smem(gemv_wide_kernel<16, false>, kGwSmemBudget);
+        if (e == cudaSuccess) e = set_smem(gemv_wide_kernel<32, true>, kGwSmemBudget);
+        if (e == cudaSuccess) e = set_smem(gemv_wide_kernel<32, false>, kGwSmemBudget);
         if (e == cudaSuccess) e = set_gemv_attrs<1>();
         if (e == cudaSuccess) e = set_gemv_attrs<2>();
         if (e == cudaSuccess) e = set_gemv_attrs<3>();
-        if (e == cudaSuccess) e = set_gemv_attrs<4>();
-        if (e == cudaSuccess) e = set_gemv_attrs<5>();
-        if (e == cudaSuccess) e = set_gemv_attrs<6>();
-        if (e == cudaSuccess) e = set_gemv_attrs<7>();
-        if (e == cudaSuccess) e = set_gemv_attrs<8>();
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8>, 2 * kMaxK);  // one row of the largest K
         if (e == cudaSuccess) e = set_smem(rmsnorm_quant_kernel<8, true>, 2 * kMaxK);
         if (e == cudaSuccess) e = set_smem(gemm_bwd_kernel<0>, BwLayout<0>::smem_bytes);
         if (e == cudaSuccess) e = set_smem(gemm_bwd_kernel<1>, BwLayout<1>::smem_bytes);
         if (e == cudaSuccess) e = set_smem(mlgru_scan_tma_kernel, kStSmemBytes);
         if (e != cudaSuccess) return MMF_ERR_CUDA;
+        // how many clusters of k CTAs of the decode tensor-core kernel (one CTA
+        // per SM) the GPU holds at once: its plan keeps a launch to one wave
+        for (int k = 1; k <= kGwMaxCluster; ++k) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(static_cast<unsigned>(k));
+            cfg.blockDim = dim3(kGwThreads);
+            cfg.dynamicSmemBytes = kGwSmemBudget;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = static_cast<unsigned>(k);
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, gemv_wide_kernel<32, true>, &cfg) != cudaSuccess) {
+                (void)cudaGetLastError();
+                n = k == 1 ? st.num_sms : 0;
+            }
+            st.wide_clusters[k] = n;
+        }
         if (!g_encode_tiled) {
             void* fn = nullptr;
             cudaDriverEntryPointQueryResult q;
@@ -142,9 +159,11 @@ mmf_status check_shape(int64_t M, int64_t K, int64_t N) {
 // Small M: up to kDecodeTcMinM - 1 tokens the CUDA-core decode kernel (its
 // add/sub cost grows with M, about M/4 integer instructions per weight); from
 // there to kDecodeTcMaxM the decode tensor-core kernel after a quantiser
-// launch (its cost is set by issuing K/32 MMAs per 128-row tile from one
-// thread, whatever M is); beyond, the large-M path.
-constexpr int64_t kDecodeTcMinM = 9;
+// launch (its cost hardly depends on M: per CTA a fixed start and cluster
+// reduction, and one MMA issue sequence per 128-wide K chunk); beyond, the
+// large-M path.  Through a 2.7B layer set (4 calls, CUDA graph) the two decode
+// kernels take 35 and 41 us at 3 tokens, 46 and 42 us at 4.
+constexpr int64_t kDecodeTcMinM = 4;
 constexpr int64_t kDecodeTcMaxM = 32;
 
 bool takes_gemv(int64_t M, int64_t K) {
@@ -155,11 +174,7 @@ bool takes_gemv(int64_t M, int64_t K) {
 
 int decode_tc_nt(int64_t M) { return M <= 16 ? 16 : 32; }
 
-bool takes_decode_tc(int64_t M, int64_t K) {
-    if (M < kDecodeTcMinM || M > kDecodeTcMaxM) return false;
-    GemvTcPlan plan;
-    return gemv_tc_plan(decode_tc_nt(M), static_cast<int>(K), 1, 148, &plan);
-}
+bool takes_decode_tc(int64_t M, int64_t) { return M >= kDecodeTcMinM && M <= kDecodeTcMaxM; }
 
 // Launches a kernel, as a programmatic dependent of the previous kernel on the
 // stream when `pdl` is set.
@@ -176,6 +191,31 @@ mmf_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = pdl ? attr : nullptr;
     cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MMF_ERR_CUDA;
+    }
+    return MMF_OK;
+}
+
+// The same, in thread-block clusters of `cluster` CTAs along x.
+template <typename... KArgs, typename... Args>
+mmf_status launch_clustered(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                            int cluster, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
     if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
         (void)cudaGetLastError();
         return MMF_ERR_CUDA;
@@ -201,7 +241,7 @@ size_t workspace_size_tc(int64_t M, int64_t K) {
     return align256(static_cast<size_t>(M) * K) + 2 * align256(4 * static_cast<size_t>(M));
 }
 
-// decode tensor-core path: the codes in the B layout of NT rows, absmax, qsum
+// decode tensor-core path: the codes in the operand layout of NT rows, absmax, qsum
 size_t workspace_size_dtc(int64_t M, int64_t K) {
     return align256(static_cast<size_t>(decode_tc_nt(M)) * K) + 2 * align256(4 * static_cast<size_t>(M));
 }
@@ -214,6 +254,61 @@ Workspace carve_dtc(void* ws, int64_t M, int64_t K) {
     w.absmax = reinterpret_cast<float*>(b + cb);
     w.qsum = reinterpret_cast<int*>(b + cb + align256(4 * static_cast<size_t>(M)));
     return w;
+}
+
+mmf_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t cols, int64_t rows,
+                     int64_t pitch, int box_cols, int box_rows, CUtensorMapSwizzle swz);
+
+// The projections (N > 0) of a decode tensor-core call.
+struct WideGroup {
+    int n = 0;
+    const uint32_t* packed[kGwMaxProj];
+    const float* scale[kGwMaxProj];
+    uint16_t* y[kGwMaxProj];
+    int64_t N[kGwMaxProj];
+    int64_t slabs() const {
+        int64_t s = 0;
+        for (int g = 0; g < n; ++g) s += (N[g] + kGwRows - 1) / kGwRows;
+        return s;
+    }
+};
+
+// The decode tensor-core contraction of a group whose codes, absmax and qsum
+// are in w (and whose partial sums and counters the quantiser has cleared).
+mmf_status launch_gemv_wide(int NT, bool fused, const WideGroup& gr, const GemvWidePlan& plan, const Workspace& w,
+                            int64_t M, int64_t K, int32_t* acc, cudaStream_t s) {
+    GemvWideParams p{};
+    GemvWideMaps maps{};
+    p.codes = w.q;
+    p.absmax = w.absmax;
+    p.qsum = w.qsum;
+    p.acc = acc;
+    p.nproj = gr.n;
+    p.M = static_cast<int>(M);
+    p.K = static_cast<int>(K);
+    p.ksplit = plan.ksplit;
+    p.chunks_per_split = plan.chunks_per_split;
+    p.slab_start[0] = 0;
+    for (int g = 0; g < gr.n; ++g) {
+        p.scale[g] = gr.scale[g];
+        p.y[g] = gr.y[g];
+        p.rows[g] = static_cast<int>(gr.N[g]);
+        p.slab_start[g + 1] = p.slab_start[g] + static_cast<int>((gr.N[g] + kGwRows - 1) / kGwRows);
+        // [N_g][K/16] words, boxes of 256 rows x one 128-wide K chunk (8 words)
+        mmf_status st = encode_2d(&maps.w[g], CU_TENSOR_MAP_DATA_TYPE_UINT32, gr.packed[g], K / 16, gr.N[g], K / 4, 8,
+                                  kGwRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (st != MMF_OK) return st;
+    }
+    // a programmatic dependent of the kernel launched just before it (which
+    // wrote the codes): only the packed weights are read before the wait; a
+    // cluster per slab, one CTA per K range
+    const dim3 grid(static_cast<unsigned>(plan.grid)), block(kGwThreads);
+    const int ks = plan.ksplit;
+    if (NT == 16)
+        return fused ? launch_clustered(gemv_wide_kernel<16, true>, grid, block, plan.smem_bytes, s, true, ks, p, maps)
+                     : launch_clustered(gemv_wide_kernel<16, false>, grid, block, plan.smem_bytes, s, true, ks, p, maps);
+    return fused ? launch_clustered(gemv_wide_kernel<32, true>, grid, block, plan.smem_bytes, s, true, ks, p, maps)
+                 : launch_clustered(gemv_wide_kernel<32, false>, grid, block, plan.smem_bytes, s, true, ks, p, maps);
 }
 
 Workspace carve(void* ws, int64_t M, int64_t K) {
@@ -311,25 +406,11 @@ mmf_status launch_gemv(const GemvParams& p, const GemvPlan& plan, cudaStream_t s
         MMF_GEMV_CASE(1)
         MMF_GEMV_CASE(2)
         MMF_GEMV_CASE(3)
-        MMF_GEMV_CASE(4)
-        MMF_GEMV_CASE(5)
-        MMF_GEMV_CASE(6)
-        MMF_GEMV_CASE(7)
-        MMF_GEMV_CASE(8)
 #undef MMF_GEMV_CASE
         default: return MMF_ERR_UNSUPPORTED_SHAPE;
     }
 }
 
-// bl_nt > 0: codes in the decode tensor-core kernel's B layout of bl_nt rows
-template <bool FUSED>
-mmf_status launch_gemv_tc(int NT, const GemvTcParams& p, const GemvTcPlan& plan, cudaStream_t s) {
-    // a programmatic dependent of the quantiser launched just before it: only
-    // the packed weights and scales (parameters) are read before the wait
-    const dim3 grid(static_cast<unsigned>(plan.grid));
-    if (NT == 16) return launch(gemv_tc_kernel<16, FUSED>, grid, dim3(kGtThreads), plan.smem_bytes, s, true, p);
-    return launch(gemv_tc_kernel<32, FUSED>, grid, dim3(kGtThreads), plan.smem_bytes, s, true, p);
-}
 
 mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_t M, int64_t K, int8_t* q,
                         float* absmax, int* qsum, cudaStream_t s, bool pdl, int num_sms,
@@ -407,31 +488,21 @@ mmf_status fwd_impl(const uint16_t* x, const float* gamma, float eps, int64_t M,
     }
     if (takes_decode_tc(M, K)) {
         const int NT = decode_tc_nt(M);
-        GemvTcPlan tplan;
-        if (!gemv_tc_plan(NT, static_cast<int>(K), R, dev->num_sms, &tplan)) return MMF_ERR_UNSUPPORTED_SHAPE;
+        WideGroup gr;
+        for (int i = 0; i < count; ++i) {
+            if (proj[i].N == 0) continue;
+            gr.packed[gr.n] = proj[i].packed;
+            gr.scale[gr.n] = proj[i].scale;
+            gr.y[gr.n] = proj[i].y;
+            gr.N[gr.n] = proj[i].N;
+            ++gr.n;
+        }
+        GemvWidePlan wplan;
+        if (!gemv_wide_plan(static_cast<int>(K), gr.slabs(), dev->wide_clusters, &wplan)) return MMF_ERR_UNSUPPORTED_SHAPE;
         Workspace w = carve_dtc(workspace, M, K);
         mmf_status st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s, pdl, dev->num_sms, u, NT);
         if (st != MMF_OK) return st;
-        GemvTcParams p{};
-        p.codes = w.q;
-        p.absmax = w.absmax;
-        p.qsum = w.qsum;
-        int g = 0;
-        p.row_start[0] = 0;
-        for (int i = 0; i < count; ++i) {
-            if (proj[i].N == 0) continue;
-            p.packed[g] = proj[i].packed;
-            p.scale[g] = proj[i].scale;
-            p.y[g] = proj[i].y;
-            p.row_start[g + 1] = p.row_start[g] + static_cast<int>(proj[i].N);
-            ++g;
-        }
-        p.nproj = g;
-        p.M = static_cast<int>(M);
-        p.K = static_cast<int>(K);
-        p.rows_per_cta = tplan.rows_per_cta;
-        p.b_slots = tplan.b_slots;
-        return launch_gemv_tc<true>(NT, p, tplan, s);
+        return launch_gemv_wide(NT, true, gr, wplan, w, M, K, nullptr, s);
     }
     Workspace w = carve(workspace, M, K);
     mmf_status st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s, pdl, dev->num_sms, u);
@@ -564,25 +635,19 @@ int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t 
     }
     if (takes_decode_tc(M, K)) {
         const int NT = decode_tc_nt(M);
-        GemvTcPlan tplan;
-        if (!gemv_tc_plan(NT, static_cast<int>(K), N, dev->num_sms, &tplan)) return MMF_ERR_UNSUPPORTED_SHAPE;
+        WideGroup gr;
+        gr.n = 1;
+        gr.packed[0] = packed;
+        gr.scale[0] = nullptr;
+        gr.y[0] = nullptr;
+        gr.N[0] = N;
+        GemvWidePlan wplan;
+        if (!gemv_wide_plan(static_cast<int>(K), gr.slabs(), dev->wide_clusters, &wplan)) return MMF_ERR_UNSUPPORTED_SHAPE;
         Workspace w = carve_dtc(workspace, M, K);
         st = launch(qsum_kernel, dim3(static_cast<unsigned>(NT)), dim3(kQuantThreads), 0, s, false, q,
                     static_cast<int>(K), M, w.qsum, w.q, NT);
         if (st != MMF_OK) return st;
-        GemvTcParams p{};
-        p.codes = w.q;
-        p.qsum = w.qsum;
-        p.packed[0] = packed;
-        p.acc = acc;
-        p.row_start[0] = 0;
-        p.row_start[1] = static_cast<int>(N);
-        p.nproj = 1;
-        p.M = static_cast<int>(M);
-        p.K = static_cast<int>(K);
-        p.rows_per_cta = tplan.rows_per_cta;
-        p.b_slots = tplan.b_slots;
-        return launch_gemv_tc<false>(NT, p, tplan, s);
+        return launch_gemv_wide(NT, false, gr, wplan, w, M, K, acc, s);
     }
     Workspace w = carve(workspace, M, K);
     st = launch(qsum_kernel, dim3(static_cast<unsigned>(M)), dim3(kQuantThreads), 0, s, false, q, static_cast<int>(K),

@@ -47,10 +47,11 @@ struct AddOp {
 };
 
 // Byte offset of codes k = 8 c8 .. 8 c8 + 7 of token m in the decode
-// tensor-core kernel's B layout for NT token rows: per 128-wide K chunk, NT
-// rows of 128 bytes in 8-row 1024-byte atoms, 16-byte units swizzled by the
-// row within the atom (the 128-byte swizzle the MMA's shared-memory
-// descriptor reads).
+// tensor-core kernel's operand layout for NT token rows: per 128-wide K
+// chunk, NT rows of 128 bytes in 8-row 1024-byte atoms, 16-byte units
+// swizzled by the row within the atom (the 128-byte swizzle the MMA's
+// shared-memory descriptor reads; the kernel copies a chunk's NT rows as the
+// first rows of its A tile).
 __host__ __device__ __forceinline__ int64_t blayout_offset(int64_t m, int c8, int NT) {
     const int kc = c8 >> 4, u = (c8 & 15) >> 1, h = c8 & 1;
     const int r = static_cast<int>(m & 7);
@@ -70,7 +71,7 @@ constexpr int64_t kQuantWarpRowMinM = 4096;       // rows from which the registe
 
 // GLU: x is the gate g of the GLU channel mixer and the row normalised is
 // p = bf16(SiLU(g) * u), formed in pass 1 and kept in place of x.
-// bl_nt > 0: the codes go to q in the B layout of NT = bl_nt token rows
+// bl_nt > 0: the codes go to q in the operand layout of NT = bl_nt token rows
 // (blayout_offset) for the decode tensor-core kernel; the grid then has
 // bl_nt CTAs and those of rows M .. bl_nt - 1 write zero codes.
 template <int WPR, bool GLU = false>
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(kQuantCtaWarps * 32) rmsnorm_quant_kernel(cons
     pdl_wait();  // x may come from the previous kernel (no-op unless launched as a dependent)
     pdl_launch_dependents();
     const int C = K >> 3;
-    if (m >= M) {  // WPR == 1: the whole warp; WPR > 1: only the padding rows of the B layout
+    if (m >= M) {  // WPR == 1: the whole warp; WPR > 1: only the padding rows of the operand layout
         if (bl_nt > 0 && m < bl_nt)
             for (int c = wr * 32 + lane; c < C; c += WPR * 32)
                 *reinterpret_cast<uint2*>(q + blayout_offset(m, c, bl_nt)) = make_uint2(0u, 0u);
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(quant_reg_warps(WPR) * 32, 2) rmsnorm_quant_re
 }
 
 // qsum only (for the contraction alone, when q is given); with bl_nt > 0 it
-// also copies the codes into the decode tensor-core kernel's B layout (grid
+// also copies the codes into the decode tensor-core kernel's operand layout (grid
 // bl_nt: rows M .. bl_nt - 1 are written as zeros and get no sum).
 __global__ void __launch_bounds__(kQuantThreads) qsum_kernel(const int8_t* __restrict__ q, int K, int64_t M,
                                                              int* __restrict__ qsum, int8_t* __restrict__ bl,

@@ -70,8 +70,8 @@ const char* mmf_version(void);
 
 /* Number of kernel launches one mmf_bitlinear_fwd_group call with `count`
  * non-empty projections of N rows in total issues for this (M, K): 1 on the
- * fused decode path (1 .. 8 tokens), 2 (quantiser + contraction) for
- * 9 .. 32 tokens, 1 + count on the large-M path; 0 for an invalid or empty
+ * fused decode path (1 .. 3 tokens), 2 (quantiser + contraction) for
+ * 4 .. 32 tokens, 1 + count on the large-M path; 0 for an invalid or empty
  * shape.  A single mmf_bitlinear_fwd is count = 1. */
 int mmf_fwd_launches(int64_t M, int64_t K, int64_t N, int count);
 
@@ -79,8 +79,8 @@ int mmf_fwd_launches(int64_t M, int64_t K, int64_t N, int count);
 size_t mmf_packed_bytes(int64_t N, int64_t K);
 
 /* Bytes of device workspace mmf_bitlinear_fwd and mmf_ternary_acc need for
- * this shape; 0 when the shape takes the fused decode path (1 .. 8 tokens),
- * which needs none.  For 9 .. 32 tokens it holds the codes in the decode
+ * this shape; 0 when the shape takes the fused decode path (1 .. 3 tokens),
+ * which needs none.  For 4 .. 32 tokens it holds the codes in the decode
  * tensor-core kernel's operand layout (16 or 32 token rows per 128-wide K
  * chunk) and the per-token absmax and code sums; for more tokens the codes in
  * row-major order and the same sums.  Depends only on (M, K, N). */

@@ -46,11 +46,12 @@ def test_library_is_sm100a_only():
 def test_sizes(L):
     assert L.mmf_packed_bytes(2560, 6912) == 2560 * 6912 // 4
     assert L.mmf_packed_bytes(-1, 128) == 0
-    # up to 8 tokens take the fused CUDA-core decode kernel: no workspace
+    # up to 3 tokens take the fused CUDA-core decode kernel: no workspace
     assert L.mmf_workspace_bytes(1, 2560, 2560) == 0
-    assert L.mmf_workspace_bytes(8, 6912, 2560) == 0
-    # 9 .. 32 tokens: the codes in the decode tensor-core kernel's operand layout
+    assert L.mmf_workspace_bytes(3, 6912, 2560) == 0
+    # 4 .. 32 tokens: the codes in the decode tensor-core kernel's operand layout
     # (16 or 32 token rows per 128-wide K chunk) + absmax + qsum, 256-byte aligned
+    assert L.mmf_workspace_bytes(4, 6912, 2560) == 16 * 6912 + 2 * 256
     assert L.mmf_workspace_bytes(9, 6912, 2560) == 16 * 6912 + 2 * 256
     # large M: int8 codes + absmax + qsum, each 256-byte aligned
     M, K = 8192, 2048
@@ -184,9 +185,10 @@ def test_shape_limits(L):
 
 
 def test_launch_counts_follow_the_path(L):
-    # up to 8 tokens: one launch; 9 .. 32 tokens: quantiser + contraction; more: quantiser + one per projection
+    # up to 3 tokens: one launch; 4 .. 32 tokens: quantiser + contraction; more: quantiser + one per projection
     assert L.mmf_fwd_launches(1, 2560, 7680, 3) == 1
-    assert L.mmf_fwd_launches(8, 2560, 7680, 3) == 1
+    assert L.mmf_fwd_launches(3, 2560, 7680, 3) == 1
+    assert L.mmf_fwd_launches(4, 2560, 7680, 3) == 2
     assert L.mmf_fwd_launches(9, 2560, 7680, 3) == 2
     assert L.mmf_fwd_launches(32, 6912, 2560, 1) == 2
     assert L.mmf_fwd_launches(33, 2560, 7680, 3) == 4
@@ -195,15 +197,15 @@ def test_launch_counts_follow_the_path(L):
 
 
 def test_workspace_sizes_follow_the_path(L):
-    # up to 8 tokens (the CUDA-core decode kernel) need none; 9 .. 32 tokens (the
+    # up to 3 tokens (the CUDA-core decode kernel) need none; 4 .. 32 tokens (the
     # decode tensor-core kernel) need the codes as 16 or 32 operand rows per K
     # chunk and the per-token absmax and code sums; the large-M path the codes,
     # absmax and sums of every token
     a256 = lambda v: (v + 255) // 256 * 256
     for K in (128, 2560, 6912):
         assert L.mmf_workspace_bytes(1, K, 256) == 0
-        assert L.mmf_workspace_bytes(8, K, 256) == 0
-        for M in (9, 16):
+        assert L.mmf_workspace_bytes(3, K, 256) == 0
+        for M in (4, 8, 9, 16):
             assert L.mmf_workspace_bytes(M, K, 256) == a256(16 * K) + 2 * a256(4 * M)
         for M in (17, 32):
             assert L.mmf_workspace_bytes(M, K, 256) == a256(32 * K) + 2 * a256(4 * M)

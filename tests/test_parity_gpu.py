@@ -3,7 +3,8 @@
 Bars: packed words, beta and int32 accumulators bit-exact; y within max
 relative error 1e-2 (floored, see gpu_cases); at most 0.1% of int8 activation
 codes differ, and then by one.  Sizes span several tiles with ragged tails on
-both kernel paths (fused decode GEMV for M <= 8, tcgen05 GEMM above), and the
+all kernel paths (fused decode GEMV for M <= 3, the decode tensor-core kernel for
+4 .. 32, the tcgen05 GEMM above), and the
 full configuration sizes are checked on sampled tokens.
 """
 import numpy as np
@@ -121,14 +122,15 @@ def test_quantize_special_rows(oracle):
 # -- ternary contraction: int32 bit-exact on the kernel's own q and packed W --------------
 
 ACC_SHAPES = [
-    # (M, K, N) CUDA-core decode kernel (1 .. 8 tokens): weight ring refilled many times per CTA
+    # (M, K, N) CUDA-core decode kernel (1 .. 3 tokens): weight ring refilled many times per CTA
     (1, 128, 1), (1, 256, 256), (1, 6912, 20000),
-    (2, 1024, 1000), (3, 2560, 333), (8, 6912, 2560), (5, 2816, 1024), (4, 4096, 9000), (2, 128, 8),
-    # decode tensor-core kernel (9 .. 32 tokens): slabs of 8 .. 128 rows, ragged slabs, the code ring
-    # refilled (K = 6912: 54 chunks), 16 and 32 operand rows
-    (9, 256, 300),
+    (2, 1024, 1000), (3, 2560, 333), (3, 6912, 2560), (2, 128, 8),
+    # decode tensor-core kernel (4 .. 32 tokens): slabs of 256 rows per projection (ragged last
+    # slab, slabs of fewer rows than 256), K split over clusters of 1 .. 8 CTAs (K = 128: one
+    # chunk; K = 6912: 54 chunks; K = 8192), 16 and 32 operand rows, one slab to several waves
+    (4, 4096, 9000), (5, 2816, 1024), (8, 6912, 2560), (9, 256, 300), (4, 128, 100),
     (16, 256, 256), (17, 384, 129), (32, 2560, 640), (32, 6912, 700), (24, 2560, 13824),
-    (31, 8192, 40000),
+    (31, 8192, 40000), (12, 1024, 80000),
     # large-M tcgen05 path: several 128-row tiles, token tiles, K stages, ragged tails
     (33, 2048, 500), (100, 1024, 257), (256, 512, 384), (300, 384, 300), (513, 2048, 200),
 ]
@@ -269,7 +271,7 @@ def test_single_token_matches_large_m_path(oracle, case):
 @pytest.mark.parametrize("K", [2560, 6912])
 def test_decode_codes_match_large_m_path(oracle, M, K):
     """The decode paths never hand their codes out: the CUDA-core kernel (up to
-    8 tokens) forms them in shared memory, the tensor-core one (9 .. 32 tokens)
+    3 tokens) forms them in shared memory, the tensor-core one (4 .. 32 tokens)
     keeps them in the MMA's operand layout with zero rows up to 16 or 32
     tokens.  M tokens on it against the same tokens as the first rows of a
     64-token batch (codes in row-major order, which the quantiser test compares
