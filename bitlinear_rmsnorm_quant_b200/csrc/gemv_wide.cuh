@@ -13,23 +13,27 @@
 // Work split: each projection of a group (sharing x) is cut into slabs of 256
 // consecutive rows (the last one partial), and each slab's K range is split
 // over the ksplit CTAs of a thread-block cluster so the SMs fill (the slabs
-// are few at decode sizes).  Each
-// CTA holds its slab's packed weights for its K range (a tensor copy of 256
-// rows per 128-wide K chunk, rows past the projection read as zero, all issued
-// before the dependency wait), unpacks them chunk by chunk into int8 B tiles
-// as they land, and streams the tokens' codes (the quantiser's operand layout: NT
-// rows of 128 B per chunk) into the first NT rows of A tiles whose other rows
-// stay zero.  The int32 accumulator sits in TMEM (128 lanes = tokens, 256
-// columns = rows).  Each CTA stages its int32 sums in shared memory (over the
-// B slots, free once its MMAs are done); after a cluster barrier every CTA of
-// the cluster forms y for its share of the slab's (token, 4-row group) items,
-// adding the ksplit CTAs' sums through distributed shared memory, and a
-// second cluster barrier keeps each CTA's sums in place until its peers have
-// read them.  Nothing goes through global memory but the weights, the codes,
-// the per-token values and y.
+// are few at decode sizes).  Each CTA holds its slab's packed weights for its
+// K range (a tensor copy of 256 rows per 128-wide K chunk, rows past the
+// projection read as zero, all issued before the dependency wait) and unpacks
+// them chunk by chunk into int8 B tiles as they land.  It takes all its
+// chunks of the tokens' codes (the quantiser's operand layout: NT rows of
+// 128 B per chunk, chunks one after the other) with one bulk copy after the
+// wait.  The A tile of chunk c is the 128-row window that starts at chunk c's
+// codes: its rows past NT are whatever follows (later chunks, the B tiles),
+// and they only reach TMEM lanes that are never read.  The int32 accumulator
+// sits in TMEM (128 lanes = tokens, 256 columns = rows).  Each CTA stages its
+// int32 sums in shared memory (over the B tiles, free once its MMAs are
+// done); after a cluster barrier every CTA of the cluster forms y for its
+// share of the slab's (token, 4-row group) items, adding the ksplit CTAs'
+// sums through distributed shared memory, and a second cluster barrier keeps
+// each CTA's sums in place until its peers have read them.  Nothing goes
+// through global memory but the weights, the codes, the per-token values and
+// y.
 // Warp roles (16 warps):
-//   warp 0      producer: weight chunks, then per chunk the codes into an A slot
-//   warp 1      TMEM allocation (256 columns); lane 0 issues the MMAs
+//   warp 0      producer: weight chunks, then the codes
+//   warp 1      TMEM allocation (256 columns); lane 0 issues the MMAs, with one
+//               barrier wait and one commit per chunk
 //   warp 2      per-token constants (code sums, dequantisation factors)
 //   warps 8-15  unpack: thread = weight row, 2-bit codes -> int8 B tile
 //   warps 0, 4, 8, 12 afterwards: tcgen05.ld of the token lanes (TMEM lanes
@@ -47,14 +51,13 @@ namespace mmf {
 constexpr int kGwRows = 256;                 // weight rows per slab (MMA N)
 constexpr int kGwThreads = 16 * 32;
 constexpr int kGwUnpackThreads = 256;        // warps 8-15, one weight row each
-constexpr int kGwASlots = 2;                 // code chunks in flight (A tiles)
-constexpr int kGwBSlots = 3;                 // unpacked weight chunks in flight (B tiles)
+constexpr int kGwSlots = 3;                  // unpacked weight chunks in flight (B tiles)
 constexpr int kGwMaxProj = 8;
 constexpr int kGwMaxChunksPerSplit = 32;     // 128-wide K chunks a CTA holds, at most
 constexpr int kGwMaxCluster = 8;             // K ranges per slab: a portable cluster
-constexpr int kGwABytes = 128 * 128;         // A tile: 128 token rows x 128 B
+constexpr int kGwAWindow = 128 * 128;        // bytes an A tile (128 rows x 128 B) spans from its start
 constexpr int kGwBBytes = kGwRows * 128;     // B tile: 256 weight rows x 128 B
-constexpr int kGwSmemBudget = 220 * 1024;
+constexpr int kGwSmemBudget = 226 * 1024;    // dynamic shared memory, within the 227 KB a CTA may hold
 
 struct GemvWideParams {
     const int8_t* codes;                      // per 128-wide K chunk, NT rows of 128 B (128-byte swizzled atoms)
@@ -82,9 +85,10 @@ struct GemvWidePlan {
     size_t smem_bytes;
 };
 
-// Shared memory: [A slots][B slots][packed weights: 256 rows x cps x 32 B]
-inline size_t gemv_wide_smem(int cps) {
-    return static_cast<size_t>(kGwASlots) * kGwABytes + static_cast<size_t>(kGwBSlots) * kGwBBytes +
+// Shared memory: [codes: cps x NT x 128 B][3 B tiles][packed weights: 256
+// rows x cps x 32 B]; the last chunk's A window reaches into the B tiles.
+inline size_t gemv_wide_smem(int cps, int NT) {
+    return static_cast<size_t>(cps) * NT * 128 + static_cast<size_t>(kGwSlots) * kGwBBytes +
            static_cast<size_t>(kGwRows) * cps * 32 + 1024;
 }
 
@@ -100,7 +104,7 @@ constexpr int kGwChunkNs = 480;
 // a piece, the piece's weights within shared memory).  clusters[k] = clusters
 // of k CTAs of this kernel that fit on the GPU at once (k = 1 .. 8).  Takes
 // the ksplit of least modelled time; false if no piece fits.
-inline bool gemv_wide_plan(int K, int64_t slabs64, const int* clusters, GemvWidePlan* plan) {
+inline bool gemv_wide_plan(int K, int NT, int64_t slabs64, const int* clusters, GemvWidePlan* plan) {
     const int nchunks = K / 128;
     if (slabs64 < 1 || nchunks < 1 || slabs64 * kGwMaxCluster > INT32_MAX) return false;
     const int slabs = static_cast<int>(slabs64);
@@ -108,7 +112,7 @@ inline bool gemv_wide_plan(int K, int64_t slabs64, const int* clusters, GemvWide
     for (int ks = 1; ks <= kGwMaxCluster && ks <= nchunks; ++ks) {
         const int cps = (nchunks + ks - 1) / ks;
         if ((nchunks + cps - 1) / cps != ks) continue;  // a piece would be empty: the smaller ksplit covers it
-        if (cps > kGwMaxChunksPerSplit || gemv_wide_smem(cps) > static_cast<size_t>(kGwSmemBudget)) continue;
+        if (cps > kGwMaxChunksPerSplit || gemv_wide_smem(cps, NT) > static_cast<size_t>(kGwSmemBudget)) continue;
         if (clusters[ks] < 1) continue;
         const int64_t waves = (slabs64 + clusters[ks] - 1) / clusters[ks];
         const int64_t t = waves * (kGwFixedNs + static_cast<int64_t>(cps) * kGwChunkNs);
@@ -121,7 +125,7 @@ inline bool gemv_wide_plan(int K, int64_t slabs64, const int* clusters, GemvWide
     if (best < 0) return false;
     plan->slabs = slabs;
     plan->grid = slabs * plan->ksplit;
-    plan->smem_bytes = gemv_wide_smem(plan->chunks_per_split);
+    plan->smem_bytes = gemv_wide_smem(plan->chunks_per_split, NT);
     return true;
 }
 
@@ -162,23 +166,24 @@ template <int NT, bool FUSED>
 __global__ void __launch_bounds__(kGwThreads, 1)
     gemv_wide_kernel(const __grid_constant__ GemvWideParams p, const __grid_constant__ GemvWideMaps maps) {
     static_assert(NT == 16 || NT == 32, "token rows of the codes: 16 or 32");
-    static_assert(NT * kGwSumStride * 4 <= kGwBSlots * kGwBBytes, "the staged sums fit the B slots");
+    static_assert(NT * kGwSumStride * 4 <= kGwSlots * kGwBBytes, "the staged sums fit the B slots");
+    static_assert(kGwAWindow - NT * 128 <= kGwSlots * kGwBBytes, "the last A window stays within the B tiles");
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t w_bar[kGwMaxChunksPerSplit];
-    __shared__ __align__(8) uint64_t a_full[kGwASlots];
-    __shared__ __align__(8) uint64_t a_empty[kGwASlots];
-    __shared__ __align__(8) uint64_t b_full[kGwBSlots];
-    __shared__ __align__(8) uint64_t b_empty[kGwBSlots];
+    __shared__ __align__(8) uint64_t codes_bar;            // all of the CTA's codes have landed
+    __shared__ __align__(8) uint64_t ready[kGwSlots];      // B tile of the slot unpacked (unpack warps)
+    __shared__ __align__(8) uint64_t slot_free[kGwSlots];  // the slot's MMAs are done (one commit)
     __shared__ __align__(8) uint64_t d_full;
     __shared__ uint32_t tmem_base_s;
-    __shared__ int abort_flag, w_issued, a_issued;
+    __shared__ int abort_flag, w_issued, codes_issued;
     __shared__ int qs_s[NT];
     __shared__ float cm_s[NT];
 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* a_base = smem;
-    uint8_t* b_base = smem + kGwASlots * kGwABytes;  // also, once this CTA's MMAs are done, its staged sums
-    uint8_t* w_s = b_base + kGwBSlots * kGwBBytes;   // chunk c: 256 rows x 32 B at w_s + c * 8 KB
+    const int cps = p.chunks_per_split;
+    uint8_t* codes_s = smem;                                   // chunk c: NT x 128 B at codes_s + c * NT * 128
+    uint8_t* b_base = smem + static_cast<size_t>(cps) * NT * 128;  // also, once the MMAs are done, the staged sums
+    uint8_t* w_s = b_base + kGwSlots * kGwBBytes;              // chunk c: 256 rows x 32 B at w_s + c * 8 KB
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nchunks = p.K >> 7;
@@ -191,8 +196,8 @@ __global__ void __launch_bounds__(kGwThreads, 1)
     const int Ng = p.rows[g];
     const int n0 = (slab - p.slab_start[g]) * kGwRows;  // the slab's first row in projection g
     const int nrows = min(Ng - n0, kGwRows);
-    const int c_lo = kr * p.chunks_per_split;
-    const int nch = min(p.chunks_per_split, nchunks - c_lo);
+    const int c_lo = kr * cps;
+    const int nch = min(cps, nchunks - c_lo);
     if (nrows <= 0 || nch <= 0) {  // the plan makes none; still meet the peers at both cluster barriers
         cluster_sync_all();
         cluster_sync_all();
@@ -201,26 +206,17 @@ __global__ void __launch_bounds__(kGwThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int c = 0; c < nch; ++c) mbar_init(&w_bar[c], 1);
-        for (int s = 0; s < kGwASlots; ++s) {
-            mbar_init(&a_full[s], 1);
-            mbar_init(&a_empty[s], 1);
-        }
-        for (int s = 0; s < kGwBSlots; ++s) {
-            mbar_init(&b_full[s], kGwUnpackThreads / 32);  // one arrival per unpack warp
-            mbar_init(&b_empty[s], 1);
+        mbar_init(&codes_bar, 1);
+        for (int s = 0; s < kGwSlots; ++s) {
+            mbar_init(&ready[s], kGwUnpackThreads / 32);  // one arrival per unpack warp
+            mbar_init(&slot_free[s], 1);
         }
         mbar_init(&d_full, 1);
         abort_flag = 0;
         w_issued = 0;
-        a_issued = 0;
+        codes_issued = 0;
         mbar_fence_init();
     }
-    // token rows past NT stay zero in every A slot (the codes fill rows 0 .. NT-1)
-    for (int i = threadIdx.x; i < kGwASlots * (128 - NT) * 8; i += kGwThreads) {
-        const int s = i / ((128 - NT) * 8), rest = i % ((128 - NT) * 8);
-        *reinterpret_cast<uint4*>(a_base + s * kGwABytes + NT * 128 + rest * 16) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    fence_proxy_async_smem();
     if (warp == 1) {
         tmem_alloc(&tmem_base_s, kGwRows);
         tmem_relinquish();
@@ -245,34 +241,30 @@ __global__ void __launch_bounds__(kGwThreads, 1)
             // the codes come from the kernel launched just before
             pdl_wait();
             pdl_launch_dependents();
-            for (int c = 0; c < nch; ++c) {
-                const int s = c % kGwASlots;
-                if (c >= kGwASlots && !mbar_wait(&a_empty[s], ((c / kGwASlots) - 1) & 1, &abort_flag)) break;
-                mbar_arrive_expect_tx(&a_full[s], NT * 128);
-                bulk_g2s(a_base + s * kGwABytes, p.codes + static_cast<size_t>(c_lo + c) * NT * 128, NT * 128,
-                         &a_full[s]);
-                a_issued = c + 1;
-            }
+            // the range's chunks are consecutive in the codes: one copy
+            mbar_arrive_expect_tx(&codes_bar, static_cast<uint32_t>(nch) * NT * 128);
+            bulk_g2s(codes_s, p.codes + static_cast<size_t>(c_lo) * NT * 128, static_cast<uint32_t>(nch) * NT * 128,
+                     &codes_bar);
+            codes_issued = 1;
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_i8(128, kGwRows);
             bool issued = false;
-            for (int c = 0; c < nch; ++c) {
-                const int sa = c % kGwASlots, sb = c % kGwBSlots;
-                if (!mbar_wait(&b_full[sb], (c / kGwBSlots) & 1, &abort_flag) ||
-                    !mbar_wait(&a_full[sa], (c / kGwASlots) & 1, &abort_flag))
-                    break;
+            const bool got_codes = mbar_wait(&codes_bar, 0, &abort_flag);
+            for (int c = 0; c < nch && got_codes; ++c) {
+                // one wait per chunk: the unpack warps' signal for its B tile
+                const int s = c % kGwSlots;
+                if (!mbar_wait(&ready[s], (c / kGwSlots) & 1, &abort_flag)) break;
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(a_base + sa * kGwABytes), b0 = smem_u32(b_base + sb * kGwBBytes);
+                const uint32_t a0 = smem_u32(codes_s + c * NT * 128), b0 = smem_u32(b_base + s * kGwBBytes);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_i8(tmem_base, sw128_kmajor_desc(a0 + 32 * kk), sw128_kmajor_desc(b0 + 32 * kk), idesc,
                            (c | kk) != 0 ? 1u : 0u);
                 issued = true;
-                mma_commit(&a_empty[sa]);
-                mma_commit(&b_empty[sb]);
+                mma_commit(&slot_free[s]);
             }
             if (issued) mma_commit(&d_full);
             if (issued && abort_flag) {  // d_full may never be waited on: let the MMAs drain here
@@ -292,9 +284,9 @@ __global__ void __launch_bounds__(kGwThreads, 1)
         const int r = threadIdx.x - 8 * 32;  // weight row of the slab, 0 .. 255 (past nrows: zeros)
         uint8_t* brow0 = b_base + (r >> 3) * 1024 + (r & 7) * 128;
         for (int c = 0; c < nch; ++c) {
-            const int sb = c % kGwBSlots;
+            const int sb = c % kGwSlots;
             bool ok = mbar_wait(&w_bar[c], 0, &abort_flag);
-            if (c >= kGwBSlots) ok = ok && mbar_wait(&b_empty[sb], ((c / kGwBSlots) - 1) & 1, &abort_flag);
+            if (c >= kGwSlots) ok = ok && mbar_wait(&slot_free[sb], ((c / kGwSlots) - 1) & 1, &abort_flag);
             if (!__all_sync(0xffffffffu, ok)) break;
             const uint4* src = reinterpret_cast<const uint4*>(w_s + c * (kGwRows * 32) + r * 32);
             const uint4 pa = src[0], pb = src[1];
@@ -311,7 +303,7 @@ __global__ void __launch_bounds__(kGwThreads, 1)
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&b_full[sb]);
+            if (lane == 0) mbar_arrive(&ready[sb]);
         }
     }
 
@@ -349,8 +341,7 @@ __global__ void __launch_bounds__(kGwThreads, 1)
         // error word is set; the slab's y is unspecified)
         int zero = 0;
         for (int c = 0; c < w_issued; ++c) mbar_wait(&w_bar[c], 0, &zero);
-        for (int u = max(0, a_issued - kGwASlots); u < a_issued; ++u)
-            mbar_wait(&a_full[u % kGwASlots], (u / kGwASlots) & 1, &zero);
+        if (codes_issued) mbar_wait(&codes_bar, 0, &zero);
     }
     // every CTA of the cluster has its sums staged
     cluster_sync_all();

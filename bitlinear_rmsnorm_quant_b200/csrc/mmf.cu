@@ -498,7 +498,7 @@ mmf_status fwd_impl(const uint16_t* x, const float* gamma, float eps, int64_t M,
             ++gr.n;
         }
         GemvWidePlan wplan;
-        if (!gemv_wide_plan(static_cast<int>(K), gr.slabs(), dev->wide_clusters, &wplan)) return MMF_ERR_UNSUPPORTED_SHAPE;
+        if (!gemv_wide_plan(static_cast<int>(K), NT, gr.slabs(), dev->wide_clusters, &wplan)) return MMF_ERR_UNSUPPORTED_SHAPE;
         Workspace w = carve_dtc(workspace, M, K);
         mmf_status st = launch_quant(x, gamma, eps, M, K, w.q, w.absmax, w.qsum, s, pdl, dev->num_sms, u, NT);
         if (st != MMF_OK) return st;
@@ -642,7 +642,7 @@ int mmf_ternary_acc(const int8_t* q, const uint32_t* packed, int64_t M, int64_t 
         gr.y[0] = nullptr;
         gr.N[0] = N;
         GemvWidePlan wplan;
-        if (!gemv_wide_plan(static_cast<int>(K), gr.slabs(), dev->wide_clusters, &wplan)) return MMF_ERR_UNSUPPORTED_SHAPE;
+        if (!gemv_wide_plan(static_cast<int>(K), NT, gr.slabs(), dev->wide_clusters, &wplan)) return MMF_ERR_UNSUPPORTED_SHAPE;
         Workspace w = carve_dtc(workspace, M, K);
         st = launch(qsum_kernel, dim3(static_cast<unsigned>(NT)), dim3(kQuantThreads), 0, s, false, q,
                     static_cast<int>(K), M, w.qsum, w.q, NT);
