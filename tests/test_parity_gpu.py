@@ -342,6 +342,7 @@ def test_training_batch_forward_sampled(oracle):
 # -- GLU channel mixer: down projection with SiLU(g) * u fused in -----------------------------
 
 @pytest.mark.parametrize("M,K,N", [(1, 6912, 2560), (3, 2816, 1024), (8, 5632, 2048), (1, 128, 16),
+                                   (16, 6912, 2560), (31, 2816, 1000),
                                    (64, 2816, 1024), (300, 6912, 640), (4100, 1024, 256)])
 def test_glu_parity(oracle, M, K, N):
     """y of the fused GLU call against the oracle's gated product fed to its BitLinear."""
@@ -556,6 +557,10 @@ def test_fwd_deterministic():
 
 @pytest.mark.parametrize("M,K,Ns", [(1, 2560, (2560, 2560, 2560, 2560)), (1, 2560, (6912, 6912)),
                                     (3, 1024, (100, 0, 333, 64)), (8, 512, (128,) * 8),
+                                    # decode tensor-core path: slabs of each projection's own, the last
+                                    # one partial, an empty projection, K split over clusters or not
+                                    (16, 2560, (2560, 100, 6912)), (5, 1024, (0, 257, 64)),
+                                    (32, 6912, (2560, 300)), (24, 128, (1000, 3)),
                                     (64, 1024, (300, 129)), (300, 384, (256, 200, 17))])
 @pytest.mark.parametrize("flags", [0, 1])
 def test_group_matches_single_calls(oracle, M, K, Ns, flags):
@@ -580,10 +585,12 @@ def test_group_matches_single_calls(oracle, M, K, Ns, flags):
         assert y_rel_error(bits_np(y), y_ref) <= Y_REL_TOL
 
 
-def test_group_pdl_chain_matches_plain():
-    """A chain of PDL launches in one stream gives the same bits as plain launches."""
+@pytest.mark.parametrize("M", [1, 16])
+def test_group_pdl_chain_matches_plain(M):
+    """A chain of PDL launches in one stream gives the same bits as plain launches
+    (one token: the fused decode kernel; 16: quantiser and tensor-core kernel)."""
     K = 2048
-    x, g, _ = make_layer(15, 1, K, 1)
+    x, g, _ = make_layer(15, M, K, 1)
     xd, gd = x.to(DEV), g.to(DEV)
     weights = []
     for i in range(6):
