@@ -21,11 +21,12 @@
 // tokens x 64 channels of f, c and g into a ring of shared-memory stages by
 // tensor copies; each of 16 compute warps takes 8 consecutive tokens of a
 // stage, computes their gates into registers and releases the stage, forms
-// its 8-token map, and after one barrier folds the stage's 16 maps in order
-// from the state entering the stage: its own incoming state on the way, the
-// state entering the next stage at the end (every warp folds the same maps in
-// the same order, so all hold the same carry).  It runs the 8 tokens from its
-// incoming state and writes o.  Needs D % 8 == 0 (16-byte row pitch for the
+// its 8-token map, and after one barrier folds the maps of the warps before
+// it, in order, from the state entering the stage: its own incoming state.
+// The last warp also applies its own map and leaves the result, the state
+// entering the next stage, in shared memory for every warp to read after the
+// next stage's barrier.  Each warp runs its 8 tokens from its incoming state
+// and writes o.  Needs D % 8 == 0 (16-byte row pitch for the
 // tensor maps) and B * T < 2^31 rows; other shapes take mlgru_scan_kernel.
 #pragma once
 #include "common.cuh"
@@ -188,6 +189,7 @@ __global__ void __launch_bounds__(kStThreads, 1) mlgru_scan_tma_kernel(const __g
     uint64_t* full = reinterpret_cast<uint64_t*>(agg + 2 * kStWarps * 32);
     uint64_t* empty = full + kStStages;
     __shared__ int abort_flag;
+    __shared__ float2 carry_sm[2][32];  // the state entering a stage, by stage parity (the last warp's)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.y;
@@ -296,18 +298,29 @@ __global__ void __launch_bounds__(kStThreads, 1) mlgru_scan_tma_kernel(const __g
         // every compute warp leaves together if any wait gave up
         if (!named_barrier_and<1, kStWarps * 32>(ok)) return;
 
-        // fold the stage's maps in order: this warp's incoming state, then the next stage's
+        // the state entering this stage: the last warp left it for stage s > 0
+        // (the barrier above orders its store before these loads)
+        if (s > 0) {
+            const float2 cv = carry_sm[s & 1][lane];
+            carry0 = cv.x;
+            carry1 = cv.y;
+        }
+        // fold the maps of the warps before this one, in order: this warp's
+        // incoming state; the last warp also applies its own map, which gives
+        // the state entering the next stage
         float h0v = carry0, h1v = carry1;
         const float4* ag = agg + (s & 1) * kStWarps * 32 + lane;
-#pragma unroll
-        for (int w = 0; w < kStWarps; ++w) {
-            if (w == warp) {
-                h0v = carry0;
-                h1v = carry1;
-            }
+#pragma unroll 4
+        for (int w = 0; w < warp; ++w) {
             const float4 m = ag[w * 32];
-            carry0 = __fmaf_rn(m.x, carry0, m.z);
-            carry1 = __fmaf_rn(m.y, carry1, m.w);
+            h0v = __fmaf_rn(m.x, h0v, m.z);
+            h1v = __fmaf_rn(m.y, h1v, m.w);
+        }
+        if (warp == kStWarps - 1) {
+            const float4 m = ag[warp * 32];
+            carry0 = __fmaf_rn(m.x, h0v, m.z);
+            carry1 = __fmaf_rn(m.y, h1v, m.w);
+            carry_sm[(s + 1) & 1][lane] = make_float2(carry0, carry1);
         }
         // the 8 tokens from the incoming state
         if (valid) {
@@ -322,7 +335,7 @@ __global__ void __launch_bounds__(kStThreads, 1) mlgru_scan_tma_kernel(const __g
             }
         }
     }
-    if (h_last && valid && warp == 0)
+    if (h_last && valid && warp == kStWarps - 1)  // the state after the last stage
         *reinterpret_cast<float2*>(h_last + static_cast<int64_t>(b) * D + k) = make_float2(carry0, carry1);
 }
 
