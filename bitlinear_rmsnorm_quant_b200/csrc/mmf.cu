@@ -423,8 +423,11 @@ mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_
         return launch(rmsnorm_quant_kernel<8>, rows_grid, dim3(256), static_cast<size_t>(K) * 2, s, pdl, x, gamma, eps,
                       static_cast<int>(K), M, q, absmax, qsum, static_cast<const uint16_t*>(nullptr), bl_nt);
     // persistent: rows in registers, WPR warps per row (K <= 2048 WPR), as many
-    // CTAs as fit on the SMs at once, never more than the rows need
-    const int wpr = static_cast<int>((K + 2047) / 2048);
+    // CTAs as fit on the SMs at once, never more than the rows need; up to
+    // K = 6912, three warps of 9 chunks a lane rather than four of 7 (3.6%
+    // faster at 8192 x 6912)
+    int wpr = static_cast<int>((K + 2047) / 2048);
+    if (wpr == 4 && K <= 3 * 32 * 9 * 8) wpr = 3;
     // 16-byte chunks a lane holds: as few as the width needs (fewer registers
     // for the row and its successor in flight)
     const int ch = static_cast<int>((K / 8 + 32 * wpr - 1) / (32 * wpr));
@@ -435,7 +438,7 @@ mmf_status launch_quant(const uint16_t* x, const float* gamma, float eps, int64_
                                                                           : rmsnorm_quant_reg_kernel<1, 8>; break;
         case 2: kern = ch <= 5 ? rmsnorm_quant_reg_kernel<2, 5> : ch <= 6 ? rmsnorm_quant_reg_kernel<2, 6>
                                                                           : rmsnorm_quant_reg_kernel<2, 8>; break;
-        case 3: kern = rmsnorm_quant_reg_kernel<3, 8>; break;
+        case 3: kern = ch <= 8 ? rmsnorm_quant_reg_kernel<3, 8> : rmsnorm_quant_reg_kernel<3, 9>; break;
         default: kern = ch <= 7 ? rmsnorm_quant_reg_kernel<4, 7> : rmsnorm_quant_reg_kernel<4, 8>; break;
     }
     const int threads = quant_reg_warps(wpr) * 32;

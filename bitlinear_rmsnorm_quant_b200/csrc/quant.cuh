@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kQuantCtaWarps * 32) rmsnorm_quant_kernel(cons
 // the definition never changes a code.  Four bytes are packed with byte
 // permutes and summed with one DP4A.  The reductions are a fixed warp tree,
 // then the group's warps in index order.
-constexpr int kQuantRegChunks = 8;       // most 16-byte chunks of x a lane holds per row (CHT)
+constexpr int kQuantRegChunks = 8;       // 16-byte chunks of x a lane holds per row (CHT), but 9 for three-warp rows
 constexpr int kMaxQuantRegK = 8192;      // WPR <= 4
 
 __host__ __device__ constexpr int quant_reg_warps(int WPR) { return WPR == 3 ? 6 : 8; }

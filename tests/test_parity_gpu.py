@@ -84,13 +84,14 @@ def test_pack_special_matrices(oracle):
 @pytest.mark.parametrize("M,K,outliers", [(16, 256, 0.0), (5, 128, 0.0), (300, 2048, 0.0), (37, 6912, 0.01),
                                           (64, 5632, 0.0),
                                           # large M: the persistent register kernel, one to four warps per
-                                          # row (K <= 2048, 4096, 6144, 8192), each lane holding as many
-                                          # 16-byte chunks as the width needs (4, 5, 6, 7 or 8), ragged
-                                          # lanes at each width
+                                          # row (K <= 2048, 4096, 6912 (three warps of up to 9 chunks),
+                                          # 8192), each lane holding as many 16-byte chunks as the width
+                                          # needs (4 .. 9), ragged lanes at each width
                                           (4100, 1024, 0.0), (5000, 128, 0.0), (4096, 1280, 0.01),
                                           (4096, 2048, 0.01), (4099, 2560, 0.01), (4100, 3072, 0.0),
                                           (4096, 4096, 0.0), (4097, 5632, 0.0), (4096, 6144, 0.01),
-                                          (4096, 6912, 0.01), (4096, 7168, 0.01), (4097, 7296, 0.0),
+                                          (4096, 6912, 0.01), (4100, 6272, 0.0), (4096, 7168, 0.01),
+                                          (4097, 7296, 0.0),
                                           (4096, 8192, 0.0),
                                           # beyond its largest K, a CTA per row
                                           (4096, 8320, 0.0), (4096, 11392, 0.01)])
