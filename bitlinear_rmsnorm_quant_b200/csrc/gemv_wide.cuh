@@ -1,12 +1,12 @@
-// gemv_wide.cuh -- decode-regime contraction for a few tokens (M <= 32) on
-// the 5th-generation tensor cores, with the weights as the MMA's wide side.
+// gemv_wide.cuh -- decode-regime contraction for a few tokens (4 <= M <= 32)
+// on the 5th-generation tensor cores, with the weights as the MMA's wide side.
 //
-// A tcgen05.mma costs the issuing thread a roughly fixed time (about 35 ns at
-// N = 16..32, about 70 ns at N = 256, where it runs at the tensor pipe's
-// peak), and every barrier wait about 100 ns.  With the tokens as N, an MMA
-// covers 128 weight rows x 32 K = 4096 weights; here the weights are the
-// N = 256 side and the tokens' codes the M = 128 side (rows past the tokens
-// are zero), so an MMA covers 256 x 32 = 8192 weights at the pipe's rate.
+// A tcgen05.mma of kind::i8 takes the tensor pipe a time that follows N x K
+// (about 28 ns at N = 16..32, about 66 ns at N = 256, K = 32, for M = 64 and
+// 128 alike), and every barrier wait costs its thread about 100 ns.  With the
+// tokens as N an MMA covers 128 weight rows x 32 K = 4096 weights; here the
+// weights are the N = 256 side and the tokens' codes the first rows of the
+// M = 128 side, so an MMA covers 256 x 32 = 8192 weights.
 // The ternary rule (ld246.com, section "三值权重的应用") is as in the other
 // kernels: codes c = w~ + 1 multiply q, and the epilogue subtracts sum q.
 //
