@@ -58,9 +58,9 @@ __host__ __device__ __forceinline__ int64_t blayout_offset(int64_t m, int c8, in
     return static_cast<int64_t>(kc) * NT * 128 + (m >> 3) * 1024 + r * 128 + ((u ^ r) << 4) + 8 * h;
 }
 
-// WPR warps per token row, one row per CTA when WPR > 1 (the library launches
-// WPR = 8: below 4096 rows, for K above the register kernel's limit, and in
-// GLU mode).  One thread brings the whole row into shared memory with bulk
+// WPR = 8 warps per token row and one row per CTA (what the library launches:
+// below 4096 rows, for K above the register kernel's limit, and in GLU mode),
+// or WPR = 1, a row per warp.  One thread brings the whole row into shared memory with bulk
 // copies (one request per row, so the row's HBM latency is paid once, not once
 // per 16-byte load); the three passes then run from shared memory, reduced
 // across the row's warps in index order.  With WPR = 1 a CTA holds one row per
@@ -83,6 +83,9 @@ __global__ void __launch_bounds__(kQuantCtaWarps * 32) rmsnorm_quant_kernel(cons
                                                                               int* __restrict__ qsum,
                                                                               const uint16_t* __restrict__ u,
                                                                               int bl_nt) {
+    // one row per CTA (WPR = 8: the reductions below share one set of slots)
+    // or one row per warp (WPR = 1: warp reductions only)
+    static_assert(WPR == 1 || WPR == kQuantCtaWarps, "one row per warp or one row per CTA");
     extern __shared__ __align__(128) uint4 xs_all[];  // one slice of K/8 chunks per row
     __shared__ __align__(8) uint64_t row_bar[kQuantCtaWarps];
     __shared__ double red_d[WPR];
