@@ -30,7 +30,6 @@ barrier and a MAX all-reduce of the device-timed step time only.
 from __future__ import annotations
 
 import argparse
-import ctypes as C
 import json
 import math
 import os
@@ -389,14 +388,11 @@ def proj_ops(M, K, N):
     return 2 * M * N * K
 
 
-def contraction_kernel(mmf, wl, api="group") -> str:
+def contraction_kernel(mmf, wl) -> str:
     """The kernel that contracts this workload's tokens with the weights, as
-    the library dispatches it: the persistent chain kernel (the whole step's
-    calls in one launch), the fused decode kernel (normalisation in the same
-    launch, no workspace), the decode tensor-core kernel (4 .. 32 tokens) or
-    the large-M tensor-core kernel."""
-    if api == "chain":
-        return "gemv_chain_kernel"
+    the library dispatches it: the fused decode kernel (normalisation in the
+    same launch, no workspace), the decode tensor-core kernel (4 .. 32 tokens)
+    or the large-M tensor-core kernel."""
     p = wl.projections[0]
     if mmf.workspace_bytes(wl.M, p.K, p.N) == 0:
         return "gemv_kernel"
@@ -496,12 +492,6 @@ class Step:
         self.bytes_per_step = 0
         self.ops_per_step = 0
         self.calls = self.make_calls(0, M, count=True)
-        if self.api == "chain":
-            # the step's calls, in the same order and with the same inputs and
-            # outputs, as one chain: one persistent launch per step
-            self.chain = mmf.Chain(self.chain_calls(), wl.eps)
-            self.calls = [(self.lib.mmf_bitlinear_chain, (C.byref(self.chain.handle),))]
-            self.launches_per_step = 1
         self.graph = None
 
     def make_calls(self, t0, t1, count=False):
@@ -532,7 +522,7 @@ class Step:
                         self.bytes_per_step += p.N * p.K // 4 + 2 * Mc * p.N + 4 + 2 * (2 * Mc * K) + 4 * K
                         self.ops_per_step += proj_ops(Mc, p.K, p.N)
                     continue
-                if self.api in ("group", "chain"):
+                if self.api == "group":
                     arr = mmf.projection_array([(self.packed[l, j], self.scales[l, j], y[j], wl.projections[j].N)
                                                 for j in js])
                     self.keep.append(arr)
@@ -558,25 +548,6 @@ class Step:
                         self.ops_per_step += proj_ops(Mc, p.K, p.N)
                     self.bytes_per_step += 2 * Mc * K + 4 * K      # x and gamma once per shared input
         return calls
-
-    def chain_calls(self):
-        """The step's calls as chain descriptors (mmf_chain_call), call for
-        call as make_calls issues them."""
-        wl = self.wl
-        out = []
-        for l in range(self.L):
-            for idx, js in sorted(self.groups.items()):
-                names = [wl.projections[j].name for j in js]
-                if self.glu and names == ["down"]:
-                    jg = [j for j, p in enumerate(wl.projections) if p.name == "gate"][0]
-                    ju = [j for j, p in enumerate(wl.projections) if p.name == "up"][0]
-                    j = js[0]
-                    out.append({"x": self.ys[l, jg], "u": self.ys[l, ju], "gamma": self.gs[l, idx],
-                                "weights": [(self.packed[l, j], self.scales[l, j], self.ys[l, j])]})
-                    continue
-                out.append({"x": self.xs[l, idx], "gamma": self.gs[l, idx],
-                            "weights": [(self.packed[l, j], self.scales[l, j], self.ys[l, j]) for j in js]})
-        return out
 
     @staticmethod
     def run(calls, stream_ptr):
@@ -743,12 +714,12 @@ def run_workload(name, args, dist, steps, warmup, peaks, peak_src, copy_gbs=None
     tokens_per_step = M * L * dist.world
     value = tokens_per_step / (ms / 1e3)
     e2e_value = tokens_per_step / (e2e_ms / 1e3)
-    kernel = contraction_kernel(st.mmf, wl, args.api)
+    kernel = contraction_kernel(st.mmf, wl)
     # the dominant kernel's own time: the step minus its quantiser launches,
     # which are timed alone in a graph of their own (none below 4 tokens, where
     # the decode kernel normalises and quantises in the same launch)
     split = None
-    if kernel not in ("gemv_kernel", "gemv_chain_kernel") and not args.glu:
+    if kernel != "gemv_kernel" and not args.glu:
         qgraph = st.capture_calls(st.quant_calls())
         q_ms, _ = st.time_graph(max(3, min(steps, 50)), 3, dist, graph=qgraph, sample_clocks=False)
         del qgraph
@@ -761,7 +732,7 @@ def run_workload(name, args, dist, steps, warmup, peaks, peak_src, copy_gbs=None
     k_ms = split["kernel_ms_per_step"] if split else ms
     k_launches = st.launches_per_step - (L * len(wl.inputs()) if split else 0)
     if hbm_bound(wl):
-        if kernel in ("gemv_kernel", "gemv_chain_kernel"):
+        if kernel == "gemv_kernel":
             k_bytes = st.bytes_per_step
             what = "packed weights, x and gamma once per shared input, y"
         else:
@@ -827,8 +798,7 @@ def run_workload(name, args, dist, steps, warmup, peaks, peak_src, copy_gbs=None
             "packed_weight_bytes": sum(p.N * p.K // 4 for p in wl.projections) * L,
             "l2": l2_note, "graph": "one CUDA graph per step",
             "parallelism": f"dp{dist.world} (token-parallel replicas)",
-            "api": {"group": "mmf_bitlinear_fwd_group", "chain": "mmf_bitlinear_chain"}.get(args.api,
-                                                                                          "mmf_bitlinear_fwd"),
+            "api": "mmf_bitlinear_fwd_group" if args.api == "group" else "mmf_bitlinear_fwd",
             "pdl": not args.no_pdl and args.api == "group", "launches_per_step": st.launches_per_step,
             "glu_down": bool(args.glu),
         },
@@ -955,9 +925,8 @@ def main(argv=None):
                     help="timed steps of each secondary workload: max(--steps, this)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-copy-kernel", action="store_true", help="skip timing mmf_hbm_copy")
-    ap.add_argument("--api", choices=("group", "single", "chain"), default="group",
-                    help="group: one call per set of projections sharing x; single: one call per projection; "
-                         "chain: the step's group calls as one chain (mmf_bitlinear_chain, 1 .. 3 tokens)")
+    ap.add_argument("--api", choices=("group", "single"), default="group",
+                    help="group: one call per set of projections sharing x; single: one call per projection")
     ap.add_argument("--glu", action="store_true",
                     help="the down projection reads the gate/up outputs through mmf_bitlinear_fwd_glu")
     ap.add_argument("--no-pdl", action="store_true", help="plain stream-ordered launches")

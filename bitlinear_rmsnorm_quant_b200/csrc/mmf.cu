@@ -7,7 +7,6 @@
 
 #include <mutex>
 #include <utility>
-#include <vector>
 
 #include "common.cuh"
 #include "copy.cuh"
@@ -19,7 +18,6 @@
 #include "scan.cuh"
 #include "bwd.cuh"
 #include "bwd_tc.cuh"
-#include "chain.cuh"
 
 namespace {
 
@@ -111,9 +109,6 @@ mmf_status device_state(DeviceState** out) {
         if (e == cudaSuccess) e = set_smem(gemm_bwd_kernel<0>, BwLayout<0>::smem_bytes);
         if (e == cudaSuccess) e = set_smem(gemm_bwd_kernel<1>, BwLayout<1>::smem_bytes);
         if (e == cudaSuccess) e = set_smem(mlgru_scan_tma_kernel, kStSmemBytes);
-        if (e == cudaSuccess) e = set_smem(gemv_chain_kernel<1>, kChainSmemBudget);
-        if (e == cudaSuccess) e = set_smem(gemv_chain_kernel<2>, kChainSmemBudget);
-        if (e == cudaSuccess) e = set_smem(gemv_chain_kernel<3>, kChainSmemBudget);
         if (e != cudaSuccess) return MMF_ERR_CUDA;
         // how many clusters of k CTAs of the decode tensor-core kernel (one CTA
         // per SM) the GPU holds at once: its plan keeps a launch to one wave
@@ -528,44 +523,6 @@ mmf_status fwd_impl(const uint16_t* x, const float* gamma, float eps, int64_t M,
         // only the quantiser may overlap the kernel before it: the contraction
         // reads the codes the quantiser writes, and waits for it either way
         if ((st = launch_tc(true, w.q, proj[i].packed, p, s, pdl, dev->num_sms)) != MMF_OK) return st;
-    }
-    return MMF_OK;
-}
-
-
-// Shape of one call of a chain on G CTAs: contiguous slabs of rows_per_cta
-// rows (a multiple of 4, the item size), cut into balanced stages that fit a
-// ring slot.
-void chain_shape(int64_t R, int K, int G, int* rows_per_cta, int* rows_per_stage) {
-    int rpc = static_cast<int>((R + G - 1) / G);
-    rpc = rpc < 4 ? 4 : (rpc + 3) & ~3;
-    const int cap = (kChainSlotBytes / (K / 4)) & ~3;  // K <= kChainMaxK: at least 16 rows
-    const int nst = (rpc + cap - 1) / cap;
-    int rps = (rpc + nst - 1) / nst;
-    rps = (rps + 3) & ~3;
-    *rows_per_cta = rpc;
-    *rows_per_stage = rps;
-}
-
-mmf_status check_chain_call(const mmf_chain_call& c, int64_t M) {
-    if (!(c.eps >= 0.0f) || c.eps > 1e30f) return MMF_ERR_INVALID_ARG;
-    if (!c.proj || c.count < 1 || c.count > MMF_MAX_GROUP) return MMF_ERR_INVALID_ARG;
-    int64_t R = 0;
-    for (int i = 0; i < c.count; ++i) {
-        if (c.proj[i].N < 0) return MMF_ERR_INVALID_ARG;
-        R += c.proj[i].N;
-    }
-    mmf_status st = check_shape(M, c.K, R);
-    if (st != MMF_OK) return st;
-    if (c.K > kChainMaxK) return MMF_ERR_UNSUPPORTED_SHAPE;
-    if (M == 0 || R == 0) return MMF_OK;  // reads and writes nothing
-    if (!c.x || !c.gamma) return MMF_ERR_INVALID_ARG;
-    if (!aligned16(c.x) || !aligned16(c.gamma) || (c.u && !aligned16(c.u))) return MMF_ERR_MISALIGNED;
-    for (int i = 0; i < c.count; ++i) {
-        if (c.proj[i].N == 0) continue;
-        if (!c.proj[i].packed || !c.proj[i].scale || !c.proj[i].y) return MMF_ERR_INVALID_ARG;
-        if (!aligned16(c.proj[i].packed) || !aligned16(c.proj[i].scale) || !aligned16(c.proj[i].y))
-            return MMF_ERR_MISALIGNED;
     }
     return MMF_OK;
 }
@@ -1004,116 +961,6 @@ int mmf_selftest_timeout(uint64_t limit_ns, int32_t* waited_out, void* stream) {
     if (st != MMF_OK) return st;
     selftest_timeout_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, waited_out);
     return launch_status();
-}
-
-size_t mmf_chain_bytes(int ncalls) {
-    if (ncalls < 1) return 0;
-    return kChainCounterBytes + static_cast<size_t>(ncalls) * sizeof(ChainCall);
-}
-
-int mmf_chain_encode(const mmf_chain_call* calls, int ncalls, int64_t M, void* buffer, size_t buffer_bytes,
-                     mmf_chain* chain) {
-    if (!chain) return MMF_ERR_INVALID_ARG;
-    *chain = mmf_chain{};
-    if (!calls || ncalls < 1 || M < 0) return MMF_ERR_INVALID_ARG;
-    if (M > kChainMaxTokens) return MMF_ERR_UNSUPPORTED_SHAPE;
-    int max_k = 0;
-    for (int i = 0; i < ncalls; ++i) {
-        const mmf_status st = check_chain_call(calls[i], M);
-        if (st != MMF_OK) return st;
-        if (calls[i].K > max_k) max_k = static_cast<int>(calls[i].K);
-    }
-    if (!buffer) return MMF_ERR_INVALID_ARG;
-    if (!aligned16(buffer)) return MMF_ERR_MISALIGNED;
-    if (buffer_bytes < mmf_chain_bytes(ncalls)) return MMF_ERR_WORKSPACE;
-    DeviceState* dev;
-    mmf_status st = device_state(&dev);
-    if (st != MMF_OK) return st;
-    const int G = dev->num_sms;
-    std::vector<ChainCall> host(static_cast<size_t>(ncalls));
-    for (int i = 0; i < ncalls; ++i) {
-        const mmf_chain_call& c = calls[i];
-        ChainCall& d = host[static_cast<size_t>(i)];
-        d = ChainCall{};
-        d.x = c.x;
-        d.u = c.u;
-        d.gamma = c.gamma;
-        d.eps = c.eps;
-        d.K = static_cast<int>(c.K);
-        int g = 0;
-        for (int j = 0; j < c.count; ++j) {
-            if (c.proj[j].N == 0) continue;
-            d.packed[g] = c.proj[j].packed;
-            d.scale[g] = c.proj[j].scale;
-            d.y[g] = c.proj[j].y;
-            d.row_start[g + 1] = d.row_start[g] + static_cast<int>(c.proj[j].N);
-            ++g;
-        }
-        d.nproj = g;
-        chain_shape(d.row_start[g], d.K, G, &d.rows_per_cta, &d.rows_per_stage);
-    }
-    uint8_t* b = static_cast<uint8_t*>(buffer);
-    if (cudaMemcpy(b + kChainCounterBytes, host.data(), host.size() * sizeof(ChainCall), cudaMemcpyHostToDevice) !=
-        cudaSuccess)
-        return MMF_ERR_CUDA;
-    const int q_bytes = static_cast<int>((M * max_k + 127) & ~int64_t(127));
-    const int gamma_bytes = 4 * max_k;
-    int slots = (kChainSmemBudget - q_bytes - gamma_bytes) / kChainSlotBytes;
-    if (slots > kChainMaxSlots) slots = kChainMaxSlots;
-    chain->buffer = buffer;
-    chain->ncalls = ncalls;
-    chain->M = static_cast<int32_t>(M);
-    chain->grid = G;
-    chain->slots = slots;
-    chain->q_bytes = q_bytes;
-    chain->gamma_bytes = gamma_bytes;
-    return MMF_OK;
-}
-
-int mmf_bitlinear_chain(const mmf_chain* chain, void* stream) {
-    if (!chain || !chain->buffer || chain->ncalls < 1) return MMF_ERR_INVALID_ARG;
-    if (chain->M < 0 || chain->M > kChainMaxTokens || chain->slots < 1 || chain->slots > kChainMaxSlots ||
-        chain->q_bytes < 0 || chain->gamma_bytes < 0 || chain->grid < 1 ||
-        static_cast<int64_t>(chain->slots) * kChainSlotBytes + chain->q_bytes + chain->gamma_bytes > kChainSmemBudget)
-        return MMF_ERR_INVALID_ARG;
-    if (chain->M == 0) return MMF_OK;
-    DeviceState* dev;
-    mmf_status st = device_state(&dev);
-    if (st != MMF_OK) return st;
-    if (chain->grid != dev->num_sms) return MMF_ERR_INVALID_ARG;  // encoded for another device
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t* b = static_cast<uint8_t*>(chain->buffer);
-    if (cudaMemsetAsync(b, 0, sizeof(unsigned), s) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return MMF_ERR_CUDA;
-    }
-    ChainParams p{};
-    p.calls = reinterpret_cast<const ChainCall*>(b + kChainCounterBytes);
-    p.counter = reinterpret_cast<unsigned*>(b);
-    p.ncalls = chain->ncalls;
-    p.M = chain->M;
-    p.slots = chain->slots;
-    p.q_bytes = chain->q_bytes;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(chain->grid));
-    cfg.blockDim = dim3(kChainThreads);
-    cfg.dynamicSmemBytes = static_cast<size_t>(chain->slots) * kChainSlotBytes + static_cast<size_t>(chain->q_bytes) +
-                           static_cast<size_t>(chain->gamma_bytes);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident together, or the launch fails
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e;
-    if (chain->M == 1) e = cudaLaunchKernelEx(&cfg, gemv_chain_kernel<1>, p);
-    else if (chain->M == 2) e = cudaLaunchKernelEx(&cfg, gemv_chain_kernel<2>, p);
-    else e = cudaLaunchKernelEx(&cfg, gemv_chain_kernel<3>, p);
-    if (e != cudaSuccess) {
-        (void)cudaGetLastError();
-        return MMF_ERR_CUDA;
-    }
-    return MMF_OK;
 }
 
 int mmf_check_async(void* stream) {

@@ -50,9 +50,6 @@ SIGNATURES = {
     "mmf_hbm_copy": (_INT, [_P, _P, _SZ, _P]),
     "mmf_selftest_timeout": (_INT, [C.c_uint64, _P, _P]),
     "mmf_check_async": (_INT, [_P]),
-    "mmf_chain_bytes": (_SZ, [_INT]),
-    "mmf_chain_encode": (_INT, [_P, _INT, _I64, _P, _SZ, _P]),
-    "mmf_bitlinear_chain": (_INT, [_P, _P]),
 }
 
 
@@ -64,17 +61,6 @@ MAX_GROUP = 8
 class Projection(C.Structure):
     """mirror of mmf_projection"""
     _fields_ = [("packed", _P), ("scale", _P), ("y", _P), ("N", _I64)]
-
-
-class ChainCall(C.Structure):
-    """mirror of mmf_chain_call"""
-    _fields_ = [("x", _P), ("u", _P), ("gamma", _P), ("eps", _F), ("K", _I64), ("proj", _P), ("count", _INT)]
-
-
-class ChainHandle(C.Structure):
-    """mirror of mmf_chain"""
-    _fields_ = [("buffer", _P), ("ncalls", C.c_int32), ("M", C.c_int32), ("grid", C.c_int32),
-                ("slots", C.c_int32), ("q_bytes", C.c_int32), ("gamma_bytes", C.c_int32)]
 
 
 class MMFError(RuntimeError):
@@ -301,44 +287,3 @@ def selftest_timeout(limit_ns: int, waited_out: torch.Tensor | None = None, stre
 
 def check_async(stream=None):
     check(lib().mmf_check_async(_stream(stream)), "mmf_check_async")
-
-
-# -- chains ---------------------------------------------------------------------
-
-class Chain:
-    """An encoded chain of small-M forward calls (mmf_chain_encode), launched
-    with run(). It keeps the device buffer and the tensors it names alive.
-
-    calls: a list of dicts with keys x, gamma, weights = [(packed, scale, y), ...]
-    and optionally u (GLU form: x is the gate g, one projection) and eps."""
-
-    def __init__(self, calls, eps: float = 1e-6):
-        L = lib()
-        if not calls:
-            raise ValueError("a chain needs at least one call")
-        x0 = calls[0]["x"]
-        M = x0.shape[0]
-        self._keep = []
-        descs = (ChainCall * len(calls))()
-        for i, c in enumerate(calls):
-            x = c["x"]
-            _dev(x, torch.bfloat16, "x")
-            u = c.get("u")
-            if u is not None:
-                _dev(u, torch.bfloat16, "u")
-            if x.shape[0] != M:
-                raise ValueError("every call of a chain has the same M")
-            K = x.shape[1]
-            arr = projection_array([(pk, sc, y, y.shape[1]) for (pk, sc, y) in c["weights"]])
-            self._keep.append((c, arr))
-            descs[i] = ChainCall(x.data_ptr(), u.data_ptr() if u is not None else None, c["gamma"].data_ptr(),
-                                 c.get("eps", eps), K, C.cast(arr, _P), len(c["weights"]))
-        self.M = M
-        n = int(L.mmf_chain_bytes(len(calls)))
-        self.buffer = torch.empty(max(n, 256), dtype=torch.uint8, device=x0.device)
-        self.handle = ChainHandle()
-        check(L.mmf_chain_encode(descs, len(calls), M, self.buffer.data_ptr(), self.buffer.numel(),
-                                 C.byref(self.handle)), "mmf_chain_encode")
-
-    def run(self, stream=None):
-        check(lib().mmf_bitlinear_chain(C.byref(self.handle), _stream(stream)), "mmf_bitlinear_chain")

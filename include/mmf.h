@@ -262,80 +262,6 @@ int mmf_bitlinear_fwd_group(const uint16_t* x, const float* gamma, float eps,
                             unsigned flags, void* stream);
 
 /*
- * A chain: a sequence of small-M fused forward calls in one persistent launch.
- *
- * Each call is what mmf_bitlinear_fwd_group computes (u == NULL) or, with
- * u != NULL and one projection, what mmf_bitlinear_fwd_glu computes (x is then
- * the gate g): RMSNorm, per-token absmax int8 codes, the ternary contraction
- * and the rescale (ld246.com, section "三值权重的应用"; jiqizhixin.com,
- * section "MatMul-free 语言模型架构"), with the same bits as those entry
- * points. A call reads its x and u only after every earlier call of the chain
- * has written all of its y, so the results are those of issuing the calls one
- * after another on the stream, and a call's x or u may be an earlier call's
- * y. One launch runs a whole decode step's sequence of dependent projections.
- * It pays one launch's fixed cost instead of one per call, and the weights of
- * later calls stream in while earlier ones compute.
- *
- * Limits: 0 <= M <= 3 tokens; each call has K a multiple of 128 and at most
- * 8192, and 1..MMF_MAX_GROUP projections (an entry with N == 0 is skipped).
- * Packed weights, scales and gamma must not be written by any call of the
- * chain (they are fetched ahead). A y written by one call must not be read as
- * x or u by the same call.
- */
-typedef struct mmf_chain_call {
-    const uint16_t* x;            /* bf16 [M][K], device; the gate g when u != NULL */
-    const uint16_t* u;            /* bf16 [M][K], device, or NULL */
-    const float* gamma;           /* fp32 [K], device */
-    float eps;                    /* RMSNorm epsilon, >= 0 */
-    int64_t K;
-    const mmf_projection* proj;   /* HOST array of `count` projections */
-    int count;                    /* 1 .. MMF_MAX_GROUP; with u != NULL, 1 */
-} mmf_chain_call;
-
-/* An encoded chain. mmf_chain_encode writes every field and
- * mmf_bitlinear_chain reads them; the caller does not modify them. */
-typedef struct mmf_chain {
-    void* buffer;      /* the device buffer holding the encoded calls */
-    int32_t ncalls;
-    int32_t M;
-    int32_t grid;      /* CTAs: the SM count of the device it was encoded on */
-    int32_t slots;     /* weight ring slots per CTA */
-    int32_t q_bytes;   /* shared memory for the codes */
-    int32_t gamma_bytes; /* shared memory for gamma */
-} mmf_chain;
-
-/* Device bytes an encoded chain of `ncalls` calls needs (0 if ncalls < 1). */
-size_t mmf_chain_bytes(int ncalls);
-
-/*
- * mmf_chain_encode -- checks the `ncalls` HOST descriptors `calls` (read
- * during the call only) and writes the chain's device form into `buffer`
- * (device memory, 16-byte aligned, at least mmf_chain_bytes(ncalls) bytes,
- * owned by the caller and kept alive while the chain is launched). The copy is
- * synchronous (cudaMemcpy), so this is not called during stream capture. The
- * pointers in the descriptors are recorded: the tensors they name stay valid
- * and in place for every launch. Fills *chain.
- * Errors: MMF_ERR_INVALID_ARG (null pointers, ncalls < 1, M < 0, bad eps or
- * count), MMF_ERR_UNSUPPORTED_SHAPE (M > 3, K outside the limits),
- * MMF_ERR_MISALIGNED, MMF_ERR_WORKSPACE (buffer too small), MMF_ERR_CUDA.
- * Nothing is written to *chain but zeros unless it returns MMF_OK.
- */
-int mmf_chain_encode(const mmf_chain_call* calls, int ncalls, int64_t M,
-                     void* buffer, size_t buffer_bytes, mmf_chain* chain);
-
-/*
- * mmf_bitlinear_chain -- runs an encoded chain on `stream`: a memset of the
- * chain's counter and one cooperative launch, one CTA per SM (capturable in a
- * CUDA graph). The launch waits for earlier work on the stream as usual. At
- * most one launch of a given buffer may be in flight at a time (they share
- * the counter). A wait that runs out (see mmf_check_async) ends the launch
- * early; y is then incomplete. M == 0 launches nothing.
- * Errors: MMF_ERR_INVALID_ARG (a handle not from mmf_chain_encode, or encoded
- * on a device with another SM count), MMF_ERR_CUDA (the launch failed).
- */
-int mmf_bitlinear_chain(const mmf_chain* chain, void* stream);
-
-/*
  * mmf_bitlinear_fwd_noalloc -- mmf_bitlinear_fwd without a caller-supplied
  * workspace; nothing on the pages corresponds to it (it is an interface
  * convenience, not part of the method).

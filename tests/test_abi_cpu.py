@@ -220,52 +220,3 @@ def test_largest_k_passes_the_shape_checks(L):
     # K = 65536 is inside the limit: the call gets as far as looking for a device
     assert L.mmf_bitlinear_fwd(A, A, 1e-6, A, A, 1, 65536, 16, A, A, 1 << 30, None) == 7
     assert L.mmf_quantize_act(A, A, 1e-6, 4096, 65536, A, A, None) == 7
-
-
-def test_chain_sizes_and_argument_errors(L):
-    """mmf_chain_bytes and the checks of mmf_chain_encode / mmf_bitlinear_chain
-    that return before any CUDA call."""
-    from bitlinear_rmsnorm_quant_b200 import mmf
-    assert L.mmf_chain_bytes(0) == 0
-    assert L.mmf_chain_bytes(-3) == 0
-    per = L.mmf_chain_bytes(2) - L.mmf_chain_bytes(1)
-    assert per > 0 and per % 16 == 0
-    assert L.mmf_chain_bytes(1) == 256 + per
-    arr = (mmf.Projection * 1)()
-    arr[0] = mmf.Projection(A, A, A, 64)
-    calls = (mmf.ChainCall * 2)()
-
-    def call(i, x=A, u=None, g=A, eps=1e-6, K=256, proj=arr, count=1):
-        calls[i] = mmf.ChainCall(x, u, g, eps, K, C.cast(proj, C.c_void_p) if proj is not None else None, count)
-
-    h = mmf.ChainHandle()
-    enc = lambda n=2, M=1, buf=A, nb=1 << 20: L.mmf_chain_encode(calls, n, M, buf, nb, C.byref(h))
-    call(0)
-    call(1)
-    assert L.mmf_chain_encode(calls, 2, 1, A, 1 << 20, None) == 1           # no handle
-    assert L.mmf_chain_encode(None, 2, 1, A, 1 << 20, C.byref(h)) == 1      # no calls
-    assert enc(n=0) == 1                                                    # ncalls 0
-    assert enc(M=-1) == 1                                                   # negative M
-    assert enc(M=4) == 2                                                    # above 3 tokens
-    call(1, K=8320)
-    assert enc() == 2                                                       # K above 8192
-    call(1, K=100)
-    assert enc() == 2                                                       # K not a multiple of 128
-    call(1, eps=-1.0)
-    assert enc() == 1                                                       # bad eps
-    call(1, count=0)
-    assert enc() == 1                                                       # empty group
-    call(1, count=9)
-    assert enc() == 1                                                       # group above the limit
-    call(1, x=None)
-    assert enc() == 1                                                       # no x
-    call(1, u=MIS)
-    assert enc() == 3                                                       # misaligned u
-    call(1)
-    assert enc(buf=None) == 1                                               # no buffer
-    assert enc(buf=MIS) == 3                                                # misaligned buffer
-    assert enc(nb=L.mmf_chain_bytes(2) - 1) == 4                            # buffer too small
-    assert h.buffer is None and h.ncalls == 0                               # untouched but zeroed
-    # launching a handle that was never encoded
-    assert L.mmf_bitlinear_chain(None, None) == 1
-    assert L.mmf_bitlinear_chain(C.byref(mmf.ChainHandle()), None) == 1
