@@ -26,6 +26,7 @@ using namespace mmf;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 constexpr int64_t kMaxK = 65536;  // the quantiser stages one bf16 row (2K bytes) in shared memory
+constexpr int64_t kMaxTokens = int64_t(65535) * 256;  // tokens per call (16,776,960)
 
 struct DeviceState {
     bool ready = false;
@@ -151,7 +152,7 @@ mmf_status check_shape(int64_t M, int64_t K, int64_t N) {
     if (M < 0 || N < 0 || K < 0) return MMF_ERR_INVALID_ARG;
     if (K < 128 || (K % 128) != 0 || K > kMaxK) return MMF_ERR_UNSUPPORTED_SHAPE;
     if (M > kMaxDim || N > kMaxDim) return MMF_ERR_UNSUPPORTED_SHAPE;
-    if (M > int64_t(65535) * 256) return MMF_ERR_UNSUPPORTED_SHAPE;  // token tiles on grid.y
+    if (M > kMaxTokens) return MMF_ERR_UNSUPPORTED_SHAPE;  // the range the header states
     if (M * K > (int64_t(1) << 40) || N * K > (int64_t(1) << 40)) return MMF_ERR_UNSUPPORTED_SHAPE;
     return MMF_OK;
 }

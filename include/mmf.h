@@ -26,7 +26,8 @@
  *     stream).  Calls are asynchronous and ordered on that stream; results
  *     are ready when the stream has reached the call.
  *   - bf16 tensors are passed as uint16_t bit patterns.
- *   - Shapes: M tokens (0 <= M < 2^31), K = d_in (128 <= K <= 65536,
+ *   - Shapes: M tokens (0 <= M <= 16,776,960 = 65535 * 256; the scan states
+ *     its own sizes), K = d_in (128 <= K <= 65536,
  *     K % 128 == 0), N = d_out (0 <= N < 2^31).  M == 0 or N == 0 is a no-op
  *     returning MMF_OK once the scalar arguments and K are valid; the buffer
  *     pointers of an empty problem are not checked and may be NULL.

@@ -172,7 +172,7 @@ def test_bwd_argument_errors(L):
 def test_shape_limits(L):
     f = L.mmf_bitlinear_fwd
     big_ws = 1 << 62  # claimed workspace size: the shape checks come first
-    # tokens beyond the grid's token-tile limit; a weight matrix beyond 2^40 elements
+    # tokens beyond the forward's stated limit (65535 * 256); a weight matrix beyond 2^40 elements
     assert f(A, A, 1e-6, A, A, 65535 * 256 + 1, 128, 16, A, A, big_ws, None) == 2
     assert f(A, A, 1e-6, A, A, 16, 65536, (1 << 24) + 16, A, A, big_ws, None) == 2
     # the allocation-free call refuses shapes whose workspace exceeds its static scratch
